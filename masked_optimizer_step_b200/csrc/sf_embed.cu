@@ -1,0 +1,197 @@
+// sf_embed.cu -- embedding-row gradient restricted to active rows.
+//
+// "Sparse-First Fine-Tuning" (tensorwirelabs.com), sections 1 and 2.2: an embedding row can
+// have a nonzero gradient only if its token occurs in the batch, so with a large vocabulary
+// the mask cuts nearly all of the table's gradient work. Row r gets G[r] = the sum of the
+// upstream gradients dY[t] over the batch positions t holding token r, and only rows the
+// conductor marks active are computed and stored.
+//
+// Two launches:
+//   embed_index_kernel  one CTA: for every token whose row is active, its slot; per-slot counts
+//                       (shared-memory atomics, exact), an exclusive scan into segment offsets,
+//                       and a scatter of token positions into their slot's segment of ws.
+//   embed_sum_kernel    persistent: one item = (active row, 256-column chunk). The CTA loads its
+//                       row's segment, sorts the positions ascending (rank sort in shared
+//                       memory, so the sum order never depends on atomics), then 8 warps each
+//                       sum every 8th token of the segment with 16-byte loads and the partial
+//                       sums are added in warp order. Active rows without tokens get zeros.
+// Traffic: dY rows of the tokens of active rows are read once per column chunk (8 KB per token
+// at H = 4096); 16 KB per active row is written.
+#include "sf_common.cuh"
+#include "sf_host.h"
+
+namespace sf {
+namespace {
+
+constexpr int kIndexThreads = 1024;
+constexpr int kSumThreads = 256;
+constexpr int kSumWarps = kSumThreads / 32;
+constexpr int kChunkCols = 256;             // 32 lanes x 8 bf16
+constexpr int kMaxTokens = 16384;
+constexpr int kMaxSlots = 49152;
+constexpr int kMaxSeg = 4096;               // positions a CTA sorts at once in shared memory
+
+// ws layout: seg_off[slot_cap + 1] int32 | perm[n_tok] int32
+__global__ void __launch_bounds__(kIndexThreads)
+embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int32_t *seg_off, int32_t *perm,
+                   uint32_t *status)
+{
+    extern __shared__ int cnt[];            // [slot_cap]
+    __shared__ int scan_scratch[33];
+    __shared__ int s_run;
+    const int cap = mk.slot_cap;
+    for (int s = threadIdx.x; s < cap; s += blockDim.x) cnt[s] = 0;
+    if (threadIdx.x == 0) s_run = 0;
+    __syncthreads();
+    bool bad = false;
+    for (int t = threadIdx.x; t < n_tok; t += blockDim.x) {
+        const int r = tok[t];
+        if (r < 0 || r >= mk.R) { bad = true; continue; }
+        if (!((mk.words[r >> 5] >> (r & 31)) & 1u)) continue;   // inactive row: dropped
+        const int s = mk.row_slot[r];
+        if (s >= 0) atomicAdd(&cnt[s], 1);
+    }
+    if (bad) set_status(status, SF_STATUS_BAD_TOKEN);
+    __syncthreads();
+    // exclusive scan of the counts, in slot order, chunk by chunk
+    for (int base = 0; base < cap; base += blockDim.x) {
+        const int s = base + threadIdx.x;
+        const int c = s < cap ? cnt[s] : 0;
+        int total;
+        const int off = block_exclusive_scan(c, scan_scratch, &total);
+        const int run = s_run;
+        if (s < cap) {
+            seg_off[s] = run + off;
+            cnt[s] = 0;                     // becomes the fill cursor
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) s_run = run + total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) seg_off[cap] = s_run;
+    __syncthreads();
+    for (int t = threadIdx.x; t < n_tok; t += blockDim.x) {
+        const int r = tok[t];
+        if (r < 0 || r >= mk.R || !((mk.words[r >> 5] >> (r & 31)) & 1u)) continue;
+        const int s = mk.row_slot[r];
+        if (s >= 0) perm[seg_off[s] + atomicAdd(&cnt[s], 1)] = t;
+    }
+}
+
+__global__ void __launch_bounds__(kSumThreads)
+embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, sf_mask mk, float *G, long long ld_g,
+                 const int32_t *seg_off, const int32_t *perm)
+{
+    __shared__ int pos[kMaxSeg];
+    __shared__ int sorted[kMaxSeg];
+    __shared__ float part[kSumWarps][kChunkCols];
+    const int n_act = mk.counts[0];
+    const int nchunks = (H + kChunkCols - 1) / kChunkCols;
+    const int total = n_act * nchunks;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const int k = item / nchunks;
+        const int chunk = item - k * nchunks;
+        const int r = mk.active_rows[k];
+        const int slot = mk.row_slot[r];
+        if (slot < 0) continue;
+        const int b0 = seg_off[slot], n = seg_off[slot + 1] - b0;
+        const int c0 = chunk * kChunkCols + lane * 8;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int sb = 0; sb < n; sb += kMaxSeg) {
+            const int m = min(kMaxSeg, n - sb);
+            for (int i = tid; i < m; i += kSumThreads) pos[i] = perm[b0 + sb + i];
+            __syncthreads();
+            // positions are distinct: rank = number of smaller ones
+            for (int i = tid; i < m; i += kSumThreads) {
+                const int p = pos[i];
+                int rank = 0;
+                for (int j = 0; j < m; ++j) rank += pos[j] < p;
+                sorted[rank] = p;
+            }
+            __syncthreads();
+            if (c0 < H) {
+                int i = warp;
+                for (; i + 3 * kSumWarps < m; i += 4 * kSumWarps) {
+                    uint4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v[u] = __ldg(reinterpret_cast<const uint4 *>(dY + (size_t)sorted[i + u * kSumWarps] * ld_dy + c0));
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t ww[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            acc[2 * e] = __fadd_rn(acc[2 * e], __uint_as_float(ww[e] << 16));
+                            acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], __uint_as_float(ww[e] & 0xFFFF0000u));
+                        }
+                    }
+                }
+                for (; i < m; i += kSumWarps) {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(dY + (size_t)sorted[i] * ld_dy + c0));
+                    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc[2 * e] = __fadd_rn(acc[2 * e], __uint_as_float(ww[e] << 16));
+                        acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], __uint_as_float(ww[e] & 0xFFFF0000u));
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        // fixed-order combination of the 8 warps' partial sums
+#pragma unroll
+        for (int e = 0; e < 8; ++e) part[warp][lane * 8 + e] = acc[e];
+        __syncthreads();
+        const int col = chunk * kChunkCols + tid;
+        if (col < H) {
+            float s = part[0][tid];
+#pragma unroll
+            for (int w = 1; w < kSumWarps; ++w) s = __fadd_rn(s, part[w][tid]);
+            G[(size_t)slot * ld_g + col] = s;
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+}  // namespace sf
+
+using namespace sf;
+
+extern "C" size_t sf_embed_grad_ws_bytes(int n_tok, int slot_cap)
+{
+    if (n_tok < 0 || slot_cap < 0) return 0;
+    const size_t b = ((size_t)slot_cap + 1 + (size_t)n_tok) * sizeof(int32_t);
+    return (b + 255) & ~(size_t)255;
+}
+
+extern "C" int sf_embed_grad(const int32_t *tokens, int n_tok, const void *dY, int H,
+                             int64_t ld_dy, const sf_mask *mk, float *G, int64_t ld_g, void *ws,
+                             size_t ws_bytes, uint32_t *dev_status, sf_stream stream)
+{
+    if (!mk || !G || H <= 0 || n_tok < 0 || (n_tok > 0 && (!tokens || !dY))) return SF_ERR_ARG;
+    int rc = check_mask(*mk);
+    if (rc != SF_OK) return rc;
+    if (n_tok > kMaxTokens || mk->slot_cap > kMaxSlots) return SF_ERR_UNSUPPORTED;
+    if ((H & 7) || ld_dy < H || (ld_dy & 7) || ld_g < H || (ld_g & 3)) return SF_ERR_ARG;
+    if ((n_tok > 0 && !aligned16(dY)) || !aligned16(G) || !aligned16(ws)) return SF_ERR_ALIGN;
+    if (!ws || ws_bytes < sf_embed_grad_ws_bytes(n_tok, mk->slot_cap)) return SF_ERR_ARG;
+    if (mk->slot_cap == 0) return SF_OK;
+    cudaStream_t st = as_stream(stream);
+    int32_t *seg_off = static_cast<int32_t *>(ws);
+    int32_t *perm = seg_off + mk->slot_cap + 1;
+    const size_t smem = (size_t)mk->slot_cap * sizeof(int);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return SF_ERR_CUDA;
+    embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, *mk, seg_off, perm, dev_status);
+    if (launch_status() != SF_OK) return SF_ERR_CUDA;
+    const int sms = sm_count();
+    if (sms <= 0) return SF_ERR_NO_DEVICE;
+    embed_sum_kernel<<<sms * 4, kSumThreads, 0, st>>>(static_cast<const uint16_t *>(dY), H, ld_dy,
+                                                      *mk, G, ld_g, seg_off, perm);
+    return launch_status();
+}

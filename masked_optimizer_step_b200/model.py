@@ -1,0 +1,181 @@
+"""A transformer's worth of sparse-first state and the four calls of one training step.
+
+"Sparse-First Fine-Tuning" (tensorwirelabs.com): a step derives per-row masks (section 2.1),
+computes the masked weight gradients (2.2) and the embedding-row gradient, and applies the
+fused update with the coupled pairs gate-up, query-output and key-value (2.3, 2.4). The down
+projection has no partner in a 7-projection layer and takes the plain (uncoupled) update.
+
+`SparseModel` owns the device state of every matrix (int8 + scale + residual weights, bf16 live
+copy, fp16 moments and fp32 gradients for slot rows, masks) and `StepPlan` holds the ABI
+argument arrays of one step, built once, so that issuing a step costs four C calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+
+import torch
+
+from . import binding as sf
+
+LLAMA_7B_LAYER = (("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+                  ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008))
+PARTNER = {"q": "o", "o": "q", "k": "v", "v": "k", "gate": "up", "up": "gate"}
+# coupling strength of each pair (section 2.4): strong for gate-up, weaker for attention pairs
+STRENGTH = {"gate": 0.6, "up": 0.6, "q": 0.4, "o": 0.4, "k": 0.4, "v": 0.4}
+# which layer input each projection reads: attention input, attention output, FFN input, FFN mid
+INPUT_OF = {"q": "x_attn", "k": "x_attn", "v": "x_attn", "o": "attn_out", "gate": "x_ffn",
+            "up": "x_ffn", "down": "ffn_mid"}
+
+
+@dataclass
+class Proj:
+    layer: int
+    name: str
+    mat: sf.Matrix
+
+
+class SparseModel:
+    """Device state of an embedding table plus n_layers x 7 projections."""
+
+    def __init__(self, n_layers: int, vocab: int = 32000, hidden: int = 4096, ffn: int = 11008,
+                 slot_frac: float = 0.03, emb_slots: int = 4096, device="cuda",
+                 layer_shapes=None):
+        self.device = device
+        shapes = layer_shapes or tuple((n, ffn if R == 11008 else hidden, ffn if C == 11008 else hidden)
+                                       for n, R, C in LLAMA_7B_LAYER)
+        self.shapes = shapes
+        self.emb = sf.Matrix(vocab, hidden, min(vocab, emb_slots), device) if vocab else None
+        self.projs: list[Proj] = []
+        for layer in range(n_layers):
+            for name, R, C in shapes:
+                cap = min(R, max(32, int(math.ceil(slot_frac * R))))
+                self.projs.append(Proj(layer, name, sf.Matrix(R, C, cap, device)))
+        self.index = {(p.layer, p.name): i for i, p in enumerate(self.projs)}
+        # all masks' counts in one contiguous block (one copy reads every mask's statistics)
+        mats = ([self.emb] if self.emb is not None else []) + [p.mat for p in self.projs]
+        self.counts = torch.zeros((len(mats), 8), dtype=torch.int32, device=device)
+        for i, m in enumerate(mats):
+            m.mask.counts = self.counts[i]
+        self.all_mats = mats
+
+    @property
+    def n_params(self) -> int:
+        return sum(m.R * m.C for m in self.all_mats)
+
+    def state_bytes(self) -> int:
+        total = 0
+        for m in self.all_mats:
+            for t in (m.q, m.s, m.delta, m.m, m.v, m.grad, m.live):
+                if t is not None:
+                    total += t.numel() * t.element_size()
+        return total
+
+    def init(self, seed: int, std: float = 0.02, stream=None):
+        """Random-init fp32 weights (seeded, on the device), quantise them, reset every mask."""
+        from . import synth
+        for i, m in enumerate(self.all_mats):
+            W = synth.device_weights_f32(m.R, m.C, seed, i, std=std, device=self.device)
+            sf.sf_quantize_init(W, m, stream)
+            sf.sf_mask_init(m.mask, stream)
+            del W
+
+    def partner_index(self, i: int) -> int:
+        """Index (in the update list, embedding first) of projection i's partner, or -1."""
+        p = self.projs[i]
+        other = PARTNER.get(p.name)
+        if other is None:
+            return -1
+        off = 1 if self.emb is not None else 0
+        return self.index[(p.layer, other)] + off
+
+
+class StepPlan:
+    """ABI argument arrays of one step over `model` for one set of input buffers.
+
+    inputs: dict with
+      tokens  int32 [n] device      (None: no embedding stage)
+      dY      bf16 [n x hidden]     upstream gradient of the embedding output
+      Y       list per projection: bf16 [T x R] forward outputs (row tracker input)
+      dX      list per projection: bf16 [T x R] upstream gradients of the outputs
+      A       list per projection: bf16 [T x C] inputs
+    """
+
+    def __init__(self, model: SparseModel, inputs: dict, embed_ws: torch.Tensor | None,
+                 threshold: float = 0.01):
+        self.model, self.inputs, self.threshold = model, inputs, threshold
+        L = sf.load()
+        self.lib = L
+        mats = model.all_mats
+        n = len(mats)
+        self.n_masks = n
+        self.mask_arr = (sf.sf_mask * n)(*[m.mask.struct() for m in mats])
+        srcs = []
+        if model.emb is not None:
+            tok = inputs["tokens"]
+            srcs.append(sf.sf_mask_src(sf.SF_SRC_TOKENS, tok.numel(), 0, tok.data_ptr()))
+        for i, p in enumerate(model.projs):
+            Y = inputs["Y"][i]
+            srcs.append(sf.sf_mask_src(sf.SF_SRC_OUTPUT_BF16, Y.shape[0], Y.stride(0), Y.data_ptr()))
+        self.src_arr = (sf.sf_mask_src * n)(*srcs)
+        probs = [sf.dw_problem(inputs["dX"][i], inputs["A"][i], p.mat.mask, p.mat.grad).c
+                 for i, p in enumerate(model.projs)]
+        self.n_dw = len(probs)
+        self.dw_arr = (sf.sf_dw_problem * len(probs))(*probs)
+        structs = []
+        if model.emb is not None:
+            structs.append(sf.matrix_struct(model.emb))
+        for i, p in enumerate(model.projs):
+            structs.append(sf.matrix_struct(p.mat, model.partner_index(i), 1.0, 0.0))
+        self.upd_arr = (sf.sf_matrix * len(structs))(*structs)
+        self.embed_ws = embed_ws
+        if model.emb is not None:
+            self.emb_mask = model.emb.mask.struct()
+
+    def set_tokens(self, tokens: torch.Tensor):
+        """Point the conductor and the embedding stage at another token batch (same length)."""
+        self.inputs["tokens"] = tokens
+        self.src_arr[0].ptr = tokens.data_ptr()
+
+    def set_coupling(self, phase_deg: float):
+        """Rotate every pair's mix: c_partner = strength * cos(phase) (section 2.4; the pages'
+        exact coefficient formula is not in the extracted text)."""
+        off = 1 if self.model.emb is not None else 0
+        c = math.cos(math.radians(phase_deg))
+        for i, p in enumerate(self.model.projs):
+            self.upd_arr[i + off].c_partner = STRENGTH.get(p.name, 0.0) * c
+
+    # the four calls of one step --------------------------------------------------------------
+    def masks(self, status, stream):
+        sf._check(self.lib.sf_mask_update(self.mask_arr, self.src_arr, self.n_masks, self.threshold,
+                                          status, stream), "sf_mask_update")
+
+    def dw(self, status, stream):
+        sf._check(self.lib.sf_masked_dw(self.dw_arr, self.n_dw, status, stream), "sf_masked_dw")
+
+    def embed(self, status, stream):
+        if self.model.emb is None:
+            return
+        tok, dY, G = self.inputs["tokens"], self.inputs["dY"], self.model.emb.grad
+        ws = self.embed_ws
+        sf._check(self.lib.sf_embed_grad(tok.data_ptr(), tok.numel(), dY.data_ptr(), dY.shape[1],
+                                         dY.stride(0), ctypes.byref(self.emb_mask), G.data_ptr(),
+                                         G.stride(0), ws.data_ptr(), ws.numel() * ws.element_size(),
+                                         status, stream), "sf_embed_grad")
+
+    def update(self, hp: sf.AdamParams, status, stream):
+        h = hp.struct()
+        sf._check(self.lib.sf_sparse_update(self.upd_arr, len(self.upd_arr), ctypes.byref(h), status,
+                                            stream), "sf_sparse_update")
+
+    def launches(self) -> int:
+        """Kernel launches one step issues (for the launch count of a timed region)."""
+        def chunks(n, k):
+            return (n + k - 1) // k
+        n_mask_batches = chunks(self.n_masks, 200)
+        n = 2 * n_mask_batches                       # accumulate + finalize per batch of masks
+        n += chunks(self.n_dw, sf.SF_DW_MAX_PER_LAUNCH)
+        n += 2 if self.model.emb is not None else 0
+        n += chunks(len(self.upd_arr), 200)
+        return n

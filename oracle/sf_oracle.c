@@ -5,14 +5,14 @@
  * baseline leg may load this library. The product (the CUDA library and its Python binding)
  * never calls it, and it shares no code, header, table or constant with the CUDA path.
  *
- * What it restates: "Sparse-First Fine-Tuning: Full-Weight Training at the Cost of the Active
- * Set" (tensorwirelabs.com, paper-sparse-first), sections 2.1 to 2.4:
+ * What it restates: the Sparse-First fine-tuning page (tensorwirelabs.com,
+ * paper-sparse-first), sections 2.1 to 2.4:
  *   - 2.1 Observing activity: the per-window charge rule and the row masks;
  *   - 2.2 Masked backward pass: dW = dX^T A, skipping all-empty 32-row tiles;
- *   - 2.3 Sparse state and int8 weights: W = s*q + delta, fp16 moments only for active rows,
+ *   - 2.3 (storage): W = s*q + delta, fp16 moments only for active rows,
  *         fused update that rebuilds the fp32 weight and writes back q, delta and live weights;
- *   - 2.4 The coupled update: each effective gradient drives a standard bias-corrected Adam
- *         step, with the weight decay scaled by cos(alpha).
+ *   - 2.4 (coupled pairs): the mixed gradient of each matrix goes through Adam with bias
+ *         correction, and weight decay carries a factor cos(alpha).
  * Code is plain loops, single threaded, slow on purpose so that it can be read against the
  * text. Where the text leaves a step open, the reading taken is stated beside the code.
  *
@@ -102,8 +102,8 @@ uint16_t orc_f32_to_f16(float f)
 /*
  * One observation window for a matrix of R rows. h[r] is the row's activity in the window
  * (its token hit count for the embedding, its output magnitude for a projection), hmax the
- * busiest row's. Per the text of section 2.1, every row's charge halves and gains half of its
- * share, share = h / hmax. Readings: an empty window (hmax == 0) gives share 0 (pure decay);
+ * busiest row's. Section 2.1 states the rule in words: the new charge is half the old one plus
+ * half the row's share of the window, share = h / hmax. Readings: an empty window (hmax == 0) gives share 0 (pure decay);
  * the share is an fp32 division; both halvings are exact, so the new charge is rounded once.
  * Row r is active while its charge is at least the threshold (0.01 on the pages), compared in
  * fp32. Bit i of words[w] is row 32*w + i.
@@ -239,8 +239,8 @@ void orc_masked_dw(int T, int R, int C, const uint16_t *dX, const uint16_t *A,
 }
 
 /*
- * Embedding-row gradient (sections 1 and 2.2): only rows of tokens present receive gradient,
- * and only active rows are kept. G[r, :] = sum of dY[t, :] over tokens t with id r, summed in
+ * Embedding-row gradient (sections 1 and 2.2): a row can only have gradient if its token is in
+ * the batch, and the mask keeps active rows only. G[r, :] = sum of dY[t, :] over tokens t with id r, summed in
  * fp64 in ascending t. Active rows with no token get zeros; inactive rows are not touched.
  * dY is n x H bf16 row-major, G is V x H fp64.
  */

@@ -1,0 +1,481 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Bars: masks, lists, counts and every untouched byte bit-exact; dW and embedding gradients within
+2e-3 of the fp64 oracle (relative, floored at 1e-3 of the matrix's largest entry); the update
+bit-exact (same fp32 operation order on both sides, 1e-6 relative allowed on W and delta, q exact
+away from rounding ties). Sections refer to "Sparse-First Fine-Tuning" (tensorwirelabs.com).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from masked_optimizer_step_b200 import binding as sf
+from masked_optimizer_step_b200 import synth
+from tests.gpu_helpers import (DEV, bf16_dev, check_slot_invariants, f32_dev, host, i32_dev,
+                               mask_host, rel_err, u32_dev)
+
+pytestmark = pytest.mark.gpu
+
+DW_TOL = 2e-3
+CANARY = np.uint32(0x7FBADBAD)          # a NaN pattern no kernel produces
+
+
+def _canary(shape):
+    return torch.from_numpy(np.full(shape, CANARY, dtype=np.uint32).view(np.int32)).to(DEV).view(torch.float32)
+
+
+# =============================================================================================
+# section 2.1: masks
+# =============================================================================================
+
+def test_conductor_matches_oracle_window_by_window(sf):
+    V, cap = 1024, 256
+    mk = sf.Mask(V, cap, DEV)
+    sf.sf_mask_init(mk)
+    status = sf.status_word()
+    charge = np.zeros(V, np.float32)
+    g = synth.rng(0, "tokens")
+    for w in range(10):
+        tok = synth.zipf_ids(g, 64, V)
+        sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_TOKENS, i32_dev(tok), n=len(tok))], 0.01, status)
+        words, _ = orc.window_tokens(charge, tok)
+        rows, tiles = orc.mask_lists(words)
+        mh = mask_host(mk)
+        assert mh["charge"].tobytes() == charge.tobytes(), f"window {w}"
+        assert np.array_equal(mh["words"], words)
+        assert np.array_equal(mh["rows"], rows) and np.array_equal(mh["tiles"], tiles)
+        check_slot_invariants(mh, cap)
+    assert host(status)[0] == 0
+    # the accumulator is left zero for the next window
+    assert not host(mk.accum).any()
+
+
+def test_conductor_empty_window_bad_ids_and_overflow(sf):
+    V, cap = 64, 2
+    mk = sf.Mask(V, cap, DEV)
+    sf.sf_mask_init(mk)
+    status = sf.status_word()
+    charge = np.zeros(V, np.float32)
+    tok = np.array([3, 3, 5, 7, 70, -1], np.int32)        # two ids out of range, 3 rows active
+    sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_TOKENS, i32_dev(tok), n=len(tok))], 0.01, status)
+    words, bad = orc.window_tokens(charge, tok)
+    mh = mask_host(mk)
+    assert bad == 2 and np.array_equal(mh["words"], words)
+    st = int(host(status)[0])
+    assert st & sf.SF_STATUS_BAD_TOKEN and st & sf.SF_STATUS_SLOT_OVERFLOW
+    assert mh["counts"][3] == 1                           # 3 active rows, 2 slots
+    check_slot_invariants(mh, cap)
+    for _ in range(3):                                    # empty windows: pure decay
+        sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_TOKENS, None, n=0)], 0.01, status)
+        orc.window_tokens(charge, [])
+        assert mask_host(mk)["charge"].tobytes() == charge.tobytes()
+
+
+@pytest.mark.parametrize("T,R", [(300, 1024), (1, 64), (2048, 4096)])
+def test_tracker_matches_oracle(sf, T, R):
+    cap = R // 4
+    mk = sf.Mask(R, cap, DEV)
+    sf.sf_mask_init(mk)
+    status = sf.status_word()
+    charge = np.zeros(R, np.float32)
+    for w in range(3):
+        g = synth.rng(2, "tracker", w, R)
+        rows = synth.scattered_rows(g, R, 0.01 + 0.02 * w)
+        Y = synth.tracker_outputs(g, T, synth.tracker_gains(R, rows))
+        sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_OUTPUT_BF16, bf16_dev(Y), n=T, ld=R)], 0.01, status)
+        words = orc.window_outputs(charge, Y)
+        mh = mask_host(mk)
+        assert mh["charge"].tobytes() == charge.tobytes()
+        assert np.array_equal(mh["words"], words)
+        r_, t_ = orc.mask_lists(words)
+        assert np.array_equal(mh["rows"], r_) and np.array_equal(mh["tiles"], t_)
+        check_slot_invariants(mh, cap)
+    assert host(status)[0] == 0
+
+
+def test_many_masks_in_one_call_and_explicit_sources(sf):
+    # several masks of different kinds and sizes in one call, each independent
+    specs = [(1024, "tokens"), (4096, "output"), (256, "words"), (512, "hits"), (11008, "output")]
+    masks, srcs, keep, ref = [], [], [], []
+    for i, (R, kind) in enumerate(specs):
+        mk = sf.Mask(R, R // 2, DEV)
+        sf.sf_mask_init(mk)
+        g = synth.rng(7, "misc", i)
+        charge = np.zeros(R, np.float32)
+        if kind == "tokens":
+            tok = synth.zipf_ids(g, 500, R)
+            t = i32_dev(tok)
+            srcs.append(sf.make_src(sf.SF_SRC_TOKENS, t, n=len(tok)))
+            words, _ = orc.window_tokens(charge, tok)
+        elif kind == "output":
+            Y = synth.tracker_outputs(g, 77, synth.tracker_gains(R, synth.scattered_rows(g, R, 0.01)))
+            t = bf16_dev(Y)
+            srcs.append(sf.make_src(sf.SF_SRC_OUTPUT_BF16, t, n=77, ld=R))
+            words = orc.window_outputs(charge, Y)
+        elif kind == "words":
+            words = synth.tiny_projection_mask(0, R)
+            t = u32_dev(words)
+            srcs.append(sf.make_src(sf.SF_SRC_WORDS, t))
+        else:
+            tok = synth.zipf_ids(g, 300, R)
+            hits = np.bincount(tok, minlength=R).astype(np.uint32)
+            t = u32_dev(hits)
+            srcs.append(sf.make_src(sf.SF_SRC_HITS_U32, t))
+            words, _ = orc.window_tokens(charge, tok)      # same counts, folded by the oracle
+        keep.append(t)
+        masks.append(mk)
+        ref.append((charge, words))
+    sf.sf_mask_update(masks, srcs, 0.01)
+    for mk, (charge, words), (R, kind) in zip(masks, ref, specs):
+        mh = mask_host(mk)
+        assert np.array_equal(mh["words"], words), kind
+        if kind != "words":
+            assert mh["charge"].tobytes() == charge.tobytes(), kind
+        else:
+            assert not mh["charge"].any()
+        check_slot_invariants(mh, R // 2)
+
+
+def test_slot_lifecycle_release_and_reuse(sf):
+    R, cap = 128, 8
+    mk = sf.Mask(R, cap, DEV)
+    sf.sf_mask_init(mk)
+    seq = [[0, 1, 2, 40], [1, 2, 3, 99, 100], [], [5, 6, 7, 8, 9, 10, 11, 12, 13], [5]]
+    prev = set()
+    for rows in seq:
+        w = synth.words_from_rows(R, rows)
+        sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_WORDS, u32_dev(w))], 0.01)
+        mh = mask_host(mk)
+        assert list(mh["rows"]) == sorted(rows)
+        check_slot_invariants(mh, cap)
+        for r in set(rows) - prev:                # fresh rows start with zero Adam steps
+            if mh["row_slot"][r] >= 0:
+                assert mh["slot_step"][mh["row_slot"][r]] == 0
+        prev = set(rows)
+
+
+# =============================================================================================
+# section 2.2: masked weight gradient
+# =============================================================================================
+
+def _dw_case(sf, T, R, C, active_rows, seed):
+    g = synth.rng(seed, "dx", T, R, C)
+    dX = synth.normal_bf16(g, (T, R))
+    A = synth.normal_bf16(synth.rng(seed, "act", T, R, C), (T, C))
+    words = synth.words_from_rows(R, active_rows)
+    cap = min(R, max(len(active_rows), 1) + 5)
+    mk = sf.Mask(R, cap, DEV)
+    sf.sf_mask_init(mk)
+    sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_WORDS, u32_dev(words))], 0.01)
+    dW = _canary((cap, C))
+    dXd, Ad = bf16_dev(dX), bf16_dev(A)
+    return dict(dX=dX, A=A, words=words, mask=mk, dW=dW, dXd=dXd, Ad=Ad, cap=cap, C=C)
+
+
+def _check_dw(case, ref=None):
+    if ref is None:
+        ref = orc.masked_dw(case["dX"], case["A"], case["words"])
+    mh = mask_host(case["mask"])
+    got = host(case["dW"])
+    used = set()
+    for r in mh["rows"]:
+        s = mh["row_slot"][r]
+        assert s >= 0
+        used.add(s)
+        err = rel_err(got[s], ref[r], 1e-3) if np.abs(ref[r]).max() > 0 else np.abs(got[s]).max()
+        assert err <= DW_TOL, (r, err)
+    for s in range(case["cap"]):
+        if s not in used:
+            assert got[s].view(np.uint32).tolist() == [int(CANARY)] * case["C"], f"slot {s} written"
+
+
+def test_masked_dw_tiny_projection(sf):
+    # W 256 x 512, T = 128: tile 0 full, tiles 3..7 empty, Bernoulli(0.03) rows elsewhere
+    words = synth.tiny_projection_mask(0, 256)
+    case = _dw_case(sf, 128, 256, 512, synth.rows_from_words(words), 0)
+    status = sf.status_word()
+    sf.sf_masked_dw([sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])], status)
+    _check_dw(case)
+    assert host(status)[0] == 0
+
+
+def test_masked_dw_ragged_grouped_and_degenerate(sf):
+    # one launch: ragged T (not a multiple of 64), ragged C (last N-tile 8 wide), a ragged last
+    # M-tile (7 active tiles), a full matrix, an all-empty mask and a zero-token problem
+    g = synth.rng(3, "rows")
+    cases = [
+        _dw_case(sf, 100, 384, 520, np.sort(g.choice(384, 40, replace=False)), 1),
+        _dw_case(sf, 200, 96, 64, np.arange(96), 2),
+        _dw_case(sf, 64, 256, 256, [], 3),
+        _dw_case(sf, 0, 64, 256, [1, 2, 63], 4),
+        _dw_case(sf, 333, 224, 1032, [0, 31, 32, 95, 96, 223], 5),
+    ]
+    status = sf.status_word()
+    sf.sf_masked_dw([sf.dw_problem(c["dXd"], c["Ad"], c["mask"], c["dW"]) for c in cases], status)
+    for c in cases:
+        _check_dw(c)
+    assert host(status)[0] == 0
+
+
+def test_masked_dw_every_tile_position(sf):
+    # each of 40 tiles active with one row, in turn spread over M-tiles: catches slot/lane mixups
+    R, C, T = 1280, 256, 96
+    rows = np.array([32 * w + (w * 7) % 32 for w in range(R // 32)])
+    case = _dw_case(sf, T, R, C, rows, 6)
+    sf.sf_masked_dw([sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])])
+    _check_dw(case)
+
+
+def test_masked_dw_deterministic(sf):
+    words = synth.tiny_projection_mask(0, 256)
+    case = _dw_case(sf, 1000, 256, 512, synth.rows_from_words(words), 8)
+    p = [sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])]
+    sf.sf_masked_dw(p)
+    a = host(case["dW"]).copy()
+    sf.sf_masked_dw(p)
+    assert a.tobytes() == host(case["dW"]).tobytes()
+
+
+# =============================================================================================
+# sections 1 / 2.2: embedding-row gradient
+# =============================================================================================
+
+@pytest.mark.parametrize("V,H,n", [(1024, 264, 700), (32000, 512, 4096)])
+def test_embed_grad_matches_oracle(sf, V, H, n):
+    g = synth.rng(1, "tokens", V)
+    tok = synth.zipf_ids(g, n, V)
+    dY = synth.normal_bf16(synth.rng(1, "dy", V), (n, H))
+    cap = min(V, 2048)
+    mk = sf.Mask(V, cap, DEV)
+    sf.sf_mask_init(mk)
+    charge = np.zeros(V, np.float32)
+    for w in range(3):                       # prior windows, then the batch itself
+        prior = synth.zipf_ids(synth.rng(1, "tokens", V, w), n, V)
+        sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_TOKENS, i32_dev(prior), n=n)], 0.01)
+        orc.window_tokens(charge, prior)
+    sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_TOKENS, i32_dev(tok), n=n)], 0.01)
+    words, _ = orc.window_tokens(charge, tok)
+    mh = mask_host(mk)
+    assert np.array_equal(mh["words"], words)
+    G = _canary((cap, H))
+    ws = torch.zeros(sf.sf_embed_grad_ws_bytes(n, cap) // 4, dtype=torch.int32, device=DEV)
+    status = sf.status_word()
+    sf.sf_embed_grad(i32_dev(tok), bf16_dev(dY), mk, G, ws, status)
+    ref = orc.embed_grad(tok, dY, V, words)
+    got = host(G)
+    used = set()
+    scale = max(np.abs(ref[mh["rows"]]).max(), 1.0)
+    for r in mh["rows"]:
+        s = mh["row_slot"][r]
+        used.add(s)
+        err = np.abs(got[s].astype(np.float64) - ref[r]) / np.maximum(np.abs(ref[r]), 1e-3 * scale)
+        assert err.max() <= DW_TOL, r
+    for s in range(cap):
+        if s not in used:
+            assert (got[s].view(np.uint32) == CANARY).all()
+    assert host(status)[0] == 0
+    # deterministic
+    G2 = _canary((cap, H))
+    sf.sf_embed_grad(i32_dev(tok), bf16_dev(dY), mk, G2, ws)
+    assert host(G2).tobytes() == got.tobytes()
+
+
+# =============================================================================================
+# sections 2.3 / 2.4: the fused sparse update
+# =============================================================================================
+
+def _state_from_oracle(sf, st: orc.MatrixState, cap: int) -> "sf.Matrix":
+    mat = sf.Matrix(st.R, st.C, cap, DEV)
+    mat.q.copy_(torch.from_numpy(st.q).to(DEV))
+    mat.s.copy_(f32_dev(st.s))
+    mat.delta.copy_(f32_dev(st.delta))
+    sf.sf_mask_init(mat.mask)
+    return mat
+
+
+def _compare_matrix(mat, st: orc.MatrixState, exact=True):
+    q, s, d = host(mat.q), host(mat.s), host(mat.delta)
+    mh = mask_host(mat.mask)
+    if exact:
+        assert q.tobytes() == st.q.tobytes()
+        assert s.tobytes() == st.s.tobytes()
+        assert d.tobytes() == st.delta.tobytes()
+    live = host(mat.live).view(np.uint16)
+    rows = synth.rows_from_words(st.words)
+    assert np.array_equal(live[rows], st.live[rows])
+    m, v, step = host(mat.m).view(np.uint16), host(mat.v).view(np.uint16), mh["slot_step"]
+    for r in rows:
+        sl = mh["row_slot"][r]
+        assert sl >= 0
+        assert np.array_equal(m[sl], st.m[r]) and np.array_equal(v[sl], st.v[r]), r
+        assert step[sl] == st.step[r]
+
+
+def _grad_rows(seed, step, R, C, scale=8.0):
+    g = synth.rng(seed, "grad", step, R, C)
+    return (g.standard_normal((R, C), dtype=np.float32) * np.float32(scale)).astype(np.float32)
+
+
+def _load_grad(mat, dense: np.ndarray):
+    """Place a dense R x C gradient into the slot-indexed buffer (rows with a slot only)."""
+    mh = mask_host(mat.mask)
+    buf = np.zeros((mat.grad.shape[0], mat.C), np.float32)
+    for r in mh["rows"]:
+        if mh["row_slot"][r] >= 0:
+            buf[mh["row_slot"][r]] = dense[r]
+    mat.grad.copy_(f32_dev(buf))
+
+
+def _set_words(sf, mats_words):
+    sf.sf_mask_update([m.mask for m, _ in mats_words],
+                      [sf.make_src(sf.SF_SRC_WORDS, u32_dev(w)) for _, w in mats_words], 0.01)
+
+
+def test_quantize_init_matches_oracle(sf):
+    W = synth.weights_f32(synth.rng(0, "weights"), 256, 512)
+    W[3] = 0.0
+    st = orc.MatrixState(W)
+    mat = sf.Matrix(256, 512, 4, DEV)
+    sf.sf_quantize_init(f32_dev(W), mat)
+    assert host(mat.q).tobytes() == st.q.tobytes()
+    assert host(mat.s).tobytes() == st.s.tobytes()
+    assert host(mat.delta).tobytes() == st.delta.tobytes()
+    assert np.array_equal(host(mat.live).view(np.uint16), synth.f32_to_bf16_bits(W))
+
+
+def test_adam_tables_match_oracle(sf):
+    hp = sf.AdamParams(t_max=3000)
+    bc1, bc2 = host(hp.bc1), host(hp.bc2)
+    for t in list(range(1, 50)) + [100, 999, 3000]:
+        assert bc1[t] == np.float32(orc.bias_correction(0.9, t))
+        assert bc2[t] == np.float32(orc.bias_correction(0.999, t))
+
+
+def test_update_tiny_projection_three_steps_bit_exact(sf):
+    R, C = 256, 512
+    W = synth.weights_f32(synth.rng(0, "weights"), R, C)
+    words = synth.tiny_projection_mask(0, R)
+    st = orc.MatrixState(W)
+    st.set_mask(words)
+    mat = _state_from_oracle(sf, st, 64)
+    _set_words(sf, [(mat, words)])
+    hp = sf.AdamParams()
+    ohp = orc.AdamHP()
+    status = sf.status_word()
+    q0, d0 = st.q.copy(), st.delta.copy()
+    for step in range(3):
+        grad = _grad_rows(0, step, R, C)
+        _load_grad(mat, grad)
+        sf.sf_sparse_update([sf.matrix_struct(mat)], hp, status)
+        orc.update(st, grad, ohp)
+        _compare_matrix(mat, st)
+    assert host(status)[0] == 0
+    inactive = np.setdiff1d(np.arange(R), synth.rows_from_words(words))
+    assert host(mat.q)[inactive].tobytes() == q0[inactive].tobytes()
+    assert host(mat.delta)[inactive].tobytes() == d0[inactive].tobytes()
+
+
+def test_update_coupled_pairs_and_changing_masks(sf):
+    # gate/up-like pair (b = 0.6) and a second pair (b = 0.4) with a rotating mix, plus an
+    # unpaired matrix; masks change between steps so slots are released and reused.
+    R, C = 128, 264
+    rng = synth.rng(11, "weights")
+    Ws = [synth.weights_f32(rng, R, C) for _ in range(5)]
+    pairs = {0: 1, 1: 0, 2: 3, 3: 2, 4: -1}
+    strength = {0: 0.6, 1: 0.6, 2: 0.4, 3: 0.4, 4: 0.0}
+    ohp = orc.AdamHP(lr=1e-3, wd=0.01 * np.cos(np.radians(28.4)), clip=40.0)
+    hp = sf.AdamParams(lr=1e-3, wd=0.01 * np.cos(np.radians(28.4)), clip=40.0)
+    sts = [orc.MatrixState(W) for W in Ws]
+    mats = [_state_from_oracle(sf, s, 48) for s in sts]
+    g = synth.rng(11, "rows")
+    status = sf.status_word()
+    for step in range(4):
+        words = [synth.words_from_rows(R, np.sort(g.choice(R, 20 + 5 * i, replace=False))) for i in range(5)]
+        if step == 2:
+            words[0] = words[1].copy()            # a and b fully overlapping
+        for st_, w in zip(sts, words):
+            st_.set_mask(w)
+        _set_words(sf, list(zip(mats, words)))
+        grads = [_grad_rows(11, 10 * step + i, R, C) for i in range(5)]
+        for m_, gr in zip(mats, grads):
+            _load_grad(m_, gr)
+        k = np.radians(36.0 * step)
+        structs = []
+        coef = []
+        for i in range(5):
+            c_self = 1.0
+            c_partner = float(np.float32(strength[i] * np.cos(k + i)))
+            coef.append((c_self, c_partner))
+            structs.append(sf.matrix_struct(mats[i], pairs[i], c_self, c_partner))
+        sf.sf_sparse_update(structs, hp, status)
+        # oracle: every matrix reads the original gradients, order is irrelevant
+        for i in range(5):
+            p = pairs[i]
+            if p >= 0:
+                orc.update(sts[i], grads[i], ohp, partner=sts[p], pg=grads[p],
+                           c_self=coef[i][0], c_partner=coef[i][1])
+            else:
+                orc.update(sts[i], grads[i], ohp)
+        for m_, s_ in zip(mats, sts):
+            _compare_matrix(m_, s_)
+    assert host(status)[0] == 0
+
+
+def test_update_wide_rows_and_overflowed_rows_untouched(sf):
+    # C = 11008 (the 7B feed-forward width) exercises several chunks per thread; slot capacity
+    # smaller than the active set: rows without a slot must not change.
+    R, C = 64, 11008
+    W = synth.weights_f32(synth.rng(5, "weights"), R, C)
+    words = synth.words_from_rows(R, [0, 5, 9, 33, 63])
+    st = orc.MatrixState(W)
+    mat = _state_from_oracle(sf, st, 3)
+    _set_words(sf, [(mat, words)])
+    mh = mask_host(mat.mask)
+    with_slot = [r for r in mh["rows"] if mh["row_slot"][r] >= 0]
+    assert len(with_slot) == 3
+    st.set_mask(synth.words_from_rows(R, with_slot))
+    hp, ohp = sf.AdamParams(), orc.AdamHP()
+    status = sf.status_word()
+    for step in range(2):
+        grad = _grad_rows(5, step, R, C)
+        _load_grad(mat, grad)
+        sf.sf_sparse_update([sf.matrix_struct(mat)], hp, status)
+        orc.update(st, grad, ohp)
+        _compare_matrix(mat, st)
+    assert int(host(status)[0]) == 0
+
+
+# =============================================================================================
+# one tiny-projection step end to end: mask -> dW -> update, three steps
+# =============================================================================================
+
+def test_tiny_projection_chain_three_steps(sf):
+    R, C, T, steps = 256, 512, 128, 3
+    W = synth.weights_f32(synth.rng(0, "weights"), R, C)
+    words = synth.tiny_projection_mask(0, R)
+    st = orc.MatrixState(W)
+    st.set_mask(words)
+    mat = sf.Matrix(R, C, 64, DEV)
+    sf.sf_mask_init(mat.mask)
+    sf.sf_quantize_init(f32_dev(W), mat)
+    _set_words(sf, [(mat, words)])
+    hp, ohp = sf.AdamParams(), orc.AdamHP()
+    status = sf.status_word()
+    q0 = host(mat.q).copy()
+    for step in range(steps):
+        dX = synth.normal_bf16(synth.rng(0, "dx", step), (T, R))
+        A = synth.normal_bf16(synth.rng(0, "act", step), (T, C))
+        sf.sf_masked_dw([sf.dw_problem(bf16_dev(dX), bf16_dev(A), mat.mask, mat.grad)], status)
+        sf.sf_sparse_update([sf.matrix_struct(mat)], hp, status)
+        orc.update(st, orc.masked_dw(dX, A, words, np.zeros((R, C))).astype(np.float32), ohp)
+    assert host(status)[0] == 0
+    rows = synth.rows_from_words(words)
+    Wg = orc.rebuild(host(mat.q), host(mat.s), host(mat.delta))
+    Wo = st.weight()
+    # the two dW differ by at most 2e-3 relative; through Adam (|u| <= ~3) that moves each step
+    # by at most lr * 4 * 2e-3
+    tol = steps * ohp.lr * 4 * DW_TOL
+    assert np.abs(Wg[rows] - Wo[rows]).max() <= tol
+    inactive = np.setdiff1d(np.arange(R), rows)
+    assert host(mat.q)[inactive].tobytes() == q0[inactive].tobytes()

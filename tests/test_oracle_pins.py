@@ -333,7 +333,7 @@ def test_bias_correction_against_exact_rational():
 
 def test_first_step_closed_form():
     # Fresh moments: m-hat = g, v-hat = g^2, so the step is -lr * g / (|g| + eps) (section 2.4:
-    # a standard Adam step with bias correction), before any fp16 rounding of stored moments.
+    # plain Adam with bias correction), before any fp16 rounding of stored moments.
     g = np.random.default_rng(12)
     R, C = 64, 48
     W0 = synth.weights_f32(g, R, C)
