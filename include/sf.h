@@ -169,6 +169,25 @@ int sf_embed_grad(const int32_t *tokens, int n_tok, const void *dY, int H, int64
                   const sf_mask *mk /* host */, float *G, int64_t ld_g,
                   void *ws, size_t ws_bytes, uint32_t *dev_status, sf_stream stream);
 
+/* ---- sf_embed_grad_noalloc: allocation-free variant of sf_embed_grad ------------------
+ * No counterpart in the paper: an operational addition. Same inputs, result and guarantees as
+ * sf_embed_grad, but without the caller's scratch buffer, for callers that must not allocate
+ * device memory themselves (a plugin whose host framework owns every device allocation, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit synchronisation). The scratch
+ * is a fixed array of SF_EMBED_NOALLOC_SCRATCH_INTS int32 (256 KiB) in the library's own device
+ * memory, present on every GPU that loads the library until the process exits; a call needs
+ * slot_cap + 1 + n_tok of them and returns SF_ERR_UNSUPPORTED beyond that. The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before any stream capture. All calls on a GPU share the array: calls that can
+ * overlap on the GPU (different streams or threads) race on it and must be ordered by the
+ * caller. This entry point allocates nothing.
+ */
+#define SF_EMBED_NOALLOC_SCRATCH_INTS 65536
+
+int sf_embed_grad_noalloc(const int32_t *tokens, int n_tok, const void *dY, int H, int64_t ld_dy,
+                          const sf_mask *mk /* host */, float *G, int64_t ld_g,
+                          uint32_t *dev_status, sf_stream stream);
+
 /* ---- sf_sparse_update: sections 2.3 and 2.4 --------------------------------------------
  * Storage of a matrix (section 2.3): W = s*q + delta with q int8 [R x C], s fp32 [R] (one scale
  * per row), delta fp32 [R x C] the full-precision residual; moments m, v fp16 [slot_cap x C]

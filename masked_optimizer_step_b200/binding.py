@@ -86,6 +86,9 @@ def load():
     L.sf_embed_grad_ws_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
     L.sf_embed_grad.argtypes = [_P, ctypes.c_int, _P, ctypes.c_int, _I64, ctypes.POINTER(sf_mask), _P,
                                 _I64, _P, ctypes.c_size_t, _P, _P]
+    L.sf_embed_grad_noalloc.argtypes = [_P, ctypes.c_int, _P, ctypes.c_int, _I64, ctypes.POINTER(sf_mask),
+                                        _P, _I64, _P, _P]
+    L.sf_embed_grad_noalloc.restype = ctypes.c_int
     L.sf_adam_tables.argtypes = [_F, _F, ctypes.c_int, _P, _P, _P]
     L.sf_sparse_update.argtypes = [ctypes.POINTER(sf_matrix), ctypes.c_int, ctypes.POINTER(sf_adam),
                                    _P, _P]
@@ -230,6 +233,16 @@ def sf_embed_grad(tokens, dY, mask: Mask, G, ws, status=None, stream=None):
     _check(load().sf_embed_grad(_ptr(tokens), n_tok, _ptr(dY), H, dY.stride(0), ctypes.byref(m), _ptr(G),
                                 G.stride(0), _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
                                 _stream(stream)), "sf_embed_grad")
+
+
+def sf_embed_grad_noalloc(tokens, dY, mask: Mask, G, status=None, stream=None):
+    """sf_embed_grad without a scratch buffer: the library's fixed per-GPU scratch is used, for
+    callers that must not allocate device memory. Calls on one GPU must not overlap."""
+    n_tok, H = dY.shape
+    m = mask.struct()
+    _check(load().sf_embed_grad_noalloc(_ptr(tokens), n_tok, _ptr(dY), H, dY.stride(0), ctypes.byref(m),
+                                        _ptr(G), G.stride(0), _ptr(status), _stream(stream)),
+           "sf_embed_grad_noalloc")
 
 
 def sf_adam_tables(beta1: float, beta2: float, t_max: int, bc1, bc2, stream=None):

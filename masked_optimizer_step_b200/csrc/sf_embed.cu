@@ -17,6 +17,8 @@
 //                       sums are added in warp order. Active rows without tokens get zeros.
 // Traffic: dY rows of the tokens of active rows are read once per column chunk (8 KB per token
 // at H = 4096); 16 KB per active row is written.
+#include <atomic>
+
 #include "sf_common.cuh"
 #include "sf_host.h"
 
@@ -181,6 +183,76 @@ extern "C" int sf_embed_grad(const int32_t *tokens, int n_tok, const void *dY, i
     if (mk->slot_cap == 0) return SF_OK;
     cudaStream_t st = as_stream(stream);
     int32_t *seg_off = static_cast<int32_t *>(ws);
+    int32_t *perm = seg_off + mk->slot_cap + 1;
+    const size_t smem = (size_t)mk->slot_cap * sizeof(int);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return SF_ERR_CUDA;
+    embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, *mk, seg_off, perm, dev_status);
+    if (launch_status() != SF_OK) return SF_ERR_CUDA;
+    const int sms = sm_count();
+    if (sms <= 0) return SF_ERR_NO_DEVICE;
+    embed_sum_kernel<<<sms * 4, kSumThreads, 0, st>>>(static_cast<const uint16_t *>(dY), H, ld_dy,
+                                                      *mk, G, ld_g, seg_off, perm);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free variant of sf_embed_grad.
+//
+// Some callers cannot hand the library a scratch buffer: they run inside a host program that
+// owns every device allocation (a plugin of a framework with its own memory pool, where a
+// foreign cudaMalloc would bypass the pool's accounting), or inside a latency-critical loop
+// where cudaMalloc's implicit device synchronisation is not acceptable. For them the scratch
+// of the embedding-row gradient lives in a fixed array in the library's own device memory.
+// The array exists once per GPU that loads the library and stays allocated until the process
+// exits; every call on that GPU uses it, so calls that overlap on the GPU (other streams, other
+// threads) race on it and must be serialised by the caller. Nothing in it has to start at zero:
+// each call writes the parts it later reads.
+// ---------------------------------------------------------------------------------------------
+namespace sf {
+namespace {
+
+constexpr int kNoAllocScratchInts = SF_EMBED_NOALLOC_SCRATCH_INTS;
+static __device__ __align__(256) int32_t g_embed_scratch[kNoAllocScratchInts];
+
+constexpr int kMaxDevices = 64;
+std::atomic<int32_t *> g_scratch_addr[kMaxDevices];
+
+// Device address of g_embed_scratch on the current device, looked up once per device (the
+// array's name in host code is only a stand-in for the symbol, not a device pointer).
+int32_t *noalloc_scratch()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    int32_t *p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_embed_scratch) != cudaSuccess || !addr) return nullptr;
+    g_scratch_addr[dev].store(static_cast<int32_t *>(addr), std::memory_order_release);
+    return static_cast<int32_t *>(addr);
+}
+
+}  // namespace
+}  // namespace sf
+
+extern "C" int sf_embed_grad_noalloc(const int32_t *tokens, int n_tok, const void *dY, int H,
+                                     int64_t ld_dy, const sf_mask *mk, float *G, int64_t ld_g,
+                                     uint32_t *dev_status, sf_stream stream)
+{
+    if (!mk || !G || H <= 0 || n_tok < 0 || (n_tok > 0 && (!tokens || !dY))) return SF_ERR_ARG;
+    int rc = check_mask(*mk);
+    if (rc != SF_OK) return rc;
+    if (n_tok > kMaxTokens || mk->slot_cap > kMaxSlots) return SF_ERR_UNSUPPORTED;
+    if ((long long)mk->slot_cap + 1 + n_tok > kNoAllocScratchInts) return SF_ERR_UNSUPPORTED;
+    if ((H & 7) || ld_dy < H || (ld_dy & 7) || ld_g < H || (ld_g & 3)) return SF_ERR_ARG;
+    if ((n_tok > 0 && !aligned16(dY)) || !aligned16(G)) return SF_ERR_ALIGN;
+    if (mk->slot_cap == 0) return SF_OK;
+    int32_t *scratch = noalloc_scratch();
+    if (!scratch) return SF_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    int32_t *seg_off = scratch;
     int32_t *perm = seg_off + mk->slot_cap + 1;
     const size_t smem = (size_t)mk->slot_cap * sizeof(int);
     if (smem > 48 * 1024 &&
