@@ -125,63 +125,16 @@ class Clocks:
 # synthetic workload
 # ---------------------------------------------------------------------------------------------
 
-def chosen_rows(layer, idx, R, kind, bank):
-    from masked_optimizer_step_b200 import synth
-    g = synth.rng(SEED, "rows", layer, idx)
-    rows = synth.scattered_rows(g, R, 0.01) if kind == "scattered" else synth.clustered_rows(g, R, 0.01)
-    if bank == 1:                              # the second bank drifts by ~5% of the chosen rows
-        g2 = synth.rng(SEED, "rows", layer, idx, 1)
-        if kind == "scattered":
-            k = max(1, int(round(0.05 * len(rows))))
-            keep = np.sort(g2.choice(len(rows), len(rows) - k, replace=False))
-            pool = np.setdiff1d(np.arange(R), rows)
-            rows = np.sort(np.concatenate([rows[keep], g2.choice(pool, k, replace=False)]))
-        else:
-            tiles = np.unique(rows // 32)
-            k = int(round(0.05 * len(tiles)))
-            if k:
-                pool = np.setdiff1d(np.arange(R // 32), tiles)
-                tiles = np.sort(np.concatenate([g2.choice(tiles, len(tiles) - k, replace=False),
-                                                g2.choice(pool, k, replace=False)]))
-                rows = (tiles[:, None] * 32 + np.arange(32)[None, :]).ravel()
-    return rows.astype(np.int64)
-
-
 def make_bank(model, T, kind, bank, device):
-    """Device-resident inputs of one step: tracker outputs, output gradients, layer inputs."""
-    import torch
     from masked_optimizer_step_b200 import synth
     from masked_optimizer_step_b200.model import INPUT_OF
-    Ys, dXs, As = [], [], []
-    layer_inputs = {}
-    hidden = 4096
-    for i, p in enumerate(model.projs):
-        R, C = p.mat.R, p.mat.C
-        key = (p.layer, INPUT_OF[p.name])
-        if key not in layer_inputs:
-            which = ("x_attn", "attn_out", "x_ffn", "ffn_mid").index(key[1])
-            layer_inputs[key] = synth.device_normal_bf16((T, C), SEED, "act", bank, p.layer, which,
-                                                         device=device)
-        As.append(layer_inputs[key])
-        gain = torch.from_numpy(synth.tracker_gains(R, chosen_rows(p.layer, i, R, kind, bank))).to(device)
-        gen = synth.device_generator(SEED, "tracker", bank, i, device=device)
-        z = torch.randn((T, R), generator=gen, device=device, dtype=torch.float32)
-        Ys.append(z.mul_(gain[None, :]).to(torch.bfloat16))
-        del z
-        dXs.append(synth.device_normal_bf16((T, R), SEED, "dx", bank, i, device=device))
-    dY = synth.device_normal_bf16((T, hidden), SEED, "dy", bank, device=device)
-    return {"Y": Ys, "dX": dXs, "A": As, "dY": dY, "tokens": None, "distinct_A": list(layer_inputs.values())}
+    projs = [(p.layer, p.name, p.mat.R, p.mat.C, INPUT_OF[p.name]) for p in model.projs]
+    return synth.step_bank(projs, T, kind, bank, SEED, device=device)
 
 
 def token_stream(n_windows, T, V=32000):
     from masked_optimizer_step_b200 import synth
-    g = synth.rng(SEED, "tokens")
-    rank_to_id = np.arange(V)
-    out = []
-    for w in range(n_windows):
-        rank_to_id = synth.drift_rank_map(g, rank_to_id, 0.01)
-        out.append(synth.zipf_ids(g, T, V, 1.1, rank_to_id))
-    return np.stack(out)
+    return synth.token_stream(SEED, n_windows, T, V)
 
 
 # ---------------------------------------------------------------------------------------------

@@ -12,10 +12,10 @@
 //     bias-corrected Adam, with a decoupled weight decay whose strength carries a cos(alpha).
 //
 // Design: one persistent launch covers every active row of every matrix of the step. A CTA of
-// 512 threads owns one row at a time: it streams the row's q, delta, gradient(s) and fp16
-// moments in with 8- and 16-byte vector loads (all coalesced), keeps the new weight in
-// registers, finds the new row absmax with a block reduction, then requantises from the
-// registers and streams q, delta, moments and the bf16 live row out. HBM-bound: per active
+// 256 threads owns one row at a time: it streams the row's q, delta, gradient(s) and fp16
+// moments in with 8- and 16-byte vector loads (all coalesced), parks the new weight in shared
+// memory, finds the new row absmax with a block reduction, then requantises and streams q,
+// delta and the bf16 live row out. Four CTAs per SM keep ~100 KB of loads in flight per SM. HBM-bound: per active
 // element it reads 1 + 4 + 4 + 2 + 2 bytes and writes 1 + 4 + 2 + 2 + 2 bytes.
 // Every floating-point step is an explicitly rounded intrinsic, in a fixed order, so results
 // are bit-reproducible and independent of the compiler's contraction choices.
@@ -25,7 +25,7 @@
 namespace sf {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
 constexpr int kMaxMatsPerLaunch = 200;
 constexpr int kMaxC = 32768;
 
@@ -57,21 +57,29 @@ struct UpdBatch {
 };
 static_assert(sizeof(UpdBatch) < 32000, "kernel parameter space");
 
-template <int CPT>   // 8-column chunks per thread; one chunk per thread fits two CTAs per SM
-__global__ void __launch_bounds__(kThreads, CPT == 1 ? 2 : 1)
+// One CTA owns one row at a time. Pass 1 streams the row's q, delta, gradient(s) and moments
+// through registers one 8-column chunk per thread per iteration, stores the new moments at once
+// and parks the new fp32 weight in shared memory (4*C bytes), so a thread needs few registers
+// and four CTAs share an SM; pass 2 requantises from shared memory.
+__global__ void __launch_bounds__(kThreads, 4)
 update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
 {
+    extern __shared__ float4 wrow4[];                 // new weights of the current row
+    float *wrow = reinterpret_cast<float *>(wrow4);
     __shared__ int s_prefix[kMaxMatsPerLaunch + 1];
     __shared__ int scan_scratch[33];
     __shared__ uint32_t max_scratch[33];
 
     const int tid = threadIdx.x;
-    {   // prefix of active-row counts over the matrices of this launch
-        const int c = tid < b.n ? b.d[tid].counts[0] : 0;
-        int total;
-        const int off = block_exclusive_scan(c, scan_scratch, &total);
-        if (tid < b.n) s_prefix[tid] = off;
-        if (tid == 0) s_prefix[b.n] = total;
+    for (int base = 0; base < b.n; base += kThreads) {   // prefix of active-row counts
+        const int i = base + tid;
+        const int c = i < b.n ? b.d[i].counts[0] : 0;
+        int tot;
+        const int off = block_exclusive_scan(c, scan_scratch, &tot);
+        const int run = base == 0 ? 0 : s_prefix[base];
+        __syncthreads();
+        if (i < b.n) s_prefix[i] = run + off;
+        if (tid == 0) s_prefix[min(base + kThreads, b.n)] = run + tot;
         __syncthreads();
     }
     const int total = s_prefix[b.n];
@@ -96,60 +104,42 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         const float bc1 = b.bc1[ti], bc2 = b.bc2[ti];
         const float sc = d.s[r];
         const int C = d.C, nchunks = C >> 3;
-        const size_t wrow = (size_t)r * C;
-        const size_t grow = (size_t)slot * C;
-        const size_t prow = (size_t)pslot * C;
+        const int8_t *qrow = d.q + (size_t)r * C;
+        const float *drow = d.delta + (size_t)r * C;
+        const float *grow = d.grad + (size_t)slot * C;
+        const float *prow = d.pgrad + (size_t)(pslot < 0 ? 0 : pslot) * C;
+        uint16_t *mrow = d.m + (size_t)slot * C;
+        uint16_t *vrow = d.v + (size_t)slot * C;
 
-        // Phase A: issue every load of this thread's chunks before any arithmetic, so that
-        // CPT x ~100 bytes per thread are in flight at once.
-        uint2 qv[CPT];
-        float4 dv[CPT][2], gv[CPT][2], pv[CPT][2];
-        uint4 mv[CPT], vv[CPT];
-#pragma unroll
-        for (int k = 0; k < CPT; ++k) {
-            const int j = tid + k * kThreads;
-            if (j < nchunks) {
-                const int c0 = j << 3;
-                qv[k] = __ldcs(reinterpret_cast<const uint2 *>(d.q + wrow + c0));
-                dv[k][0] = __ldcs(reinterpret_cast<const float4 *>(d.delta + wrow + c0));
-                dv[k][1] = __ldcs(reinterpret_cast<const float4 *>(d.delta + wrow + c0 + 4));
-                gv[k][0] = __ldcs(reinterpret_cast<const float4 *>(d.grad + grow + c0));
-                gv[k][1] = __ldcs(reinterpret_cast<const float4 *>(d.grad + grow + c0 + 4));
-                if (pslot >= 0) {
-                    pv[k][0] = __ldg(reinterpret_cast<const float4 *>(d.pgrad + prow + c0));
-                    pv[k][1] = __ldg(reinterpret_cast<const float4 *>(d.pgrad + prow + c0 + 4));
-                } else {
-                    pv[k][0] = pv[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-                if (t_old > 0) {
-                    mv[k] = __ldcs(reinterpret_cast<const uint4 *>(d.m + grow + c0));
-                    vv[k] = __ldcs(reinterpret_cast<const uint4 *>(d.v + grow + c0));
-                } else {
-                    mv[k] = vv[k] = make_uint4(0u, 0u, 0u, 0u);
-                }
-            }
-        }
-
-        // Phase B: rebuild, mix, Adam; moments go out at once, the new weight stays in registers.
-        float w[CPT][8];
+        // ---- pass 1: rebuild, mix, Adam; moments out, new weight to shared memory ----
         float amax = 0.0f;
-#pragma unroll
-        for (int k = 0; k < CPT; ++k) {
-            const int j = tid + k * kThreads;
-            if (j >= nchunks) continue;
+        for (int j = tid; j < nchunks; j += kThreads) {
             const int c0 = j << 3;
-            const float dl[8] = {dv[k][0].x, dv[k][0].y, dv[k][0].z, dv[k][0].w,
-                                 dv[k][1].x, dv[k][1].y, dv[k][1].z, dv[k][1].w};
-            const float ga_[8] = {gv[k][0].x, gv[k][0].y, gv[k][0].z, gv[k][0].w,
-                                  gv[k][1].x, gv[k][1].y, gv[k][1].z, gv[k][1].w};
-            const float gb_[8] = {pv[k][0].x, pv[k][0].y, pv[k][0].z, pv[k][0].w,
-                                  pv[k][1].x, pv[k][1].y, pv[k][1].z, pv[k][1].w};
-            const uint32_t mw[4] = {mv[k].x, mv[k].y, mv[k].z, mv[k].w};
-            const uint32_t vw[4] = {vv[k].x, vv[k].y, vv[k].z, vv[k].w};
+            const uint2 qv = __ldcs(reinterpret_cast<const uint2 *>(qrow + c0));
+            const float4 d0 = __ldcs(reinterpret_cast<const float4 *>(drow + c0));
+            const float4 d1 = __ldcs(reinterpret_cast<const float4 *>(drow + c0 + 4));
+            const float4 g0 = __ldcs(reinterpret_cast<const float4 *>(grow + c0));
+            const float4 g1 = __ldcs(reinterpret_cast<const float4 *>(grow + c0 + 4));
+            float4 p0 = make_float4(0.f, 0.f, 0.f, 0.f), p1 = p0;
+            if (pslot >= 0) {
+                p0 = __ldg(reinterpret_cast<const float4 *>(prow + c0));
+                p1 = __ldg(reinterpret_cast<const float4 *>(prow + c0 + 4));
+            }
+            uint4 mv = make_uint4(0u, 0u, 0u, 0u), vv = mv;
+            if (t_old > 0) {
+                mv = __ldcs(reinterpret_cast<const uint4 *>(mrow + c0));
+                vv = __ldcs(reinterpret_cast<const uint4 *>(vrow + c0));
+            }
+            const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+            const float ga_[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            const float gb_[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
+            const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
             uint32_t mout[4], vout[4];
+            float wn[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int8_t qe = static_cast<int8_t>(((e < 4 ? qv[k].x : qv[k].y) >> (8 * (e & 3))) & 0xFF);
+                const int8_t qe = static_cast<int8_t>(((e < 4 ? qv.x : qv.y) >> (8 * (e & 3))) & 0xFF);
                 const float W = __fmaf_rn(sc, (float)qe, dl[e]);
                 float ga = ga_[e], gb = gb_[e];
                 if (b.clip > 0.0f) {
@@ -157,10 +147,8 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
                     gb = fminf(fmaxf(gb, -b.clip), b.clip);
                 }
                 const float gt = __fmaf_rn(d.c_partner, gb, __fmul_rn(d.c_self, ga));
-                const uint16_t mh = (uint16_t)(mw[e >> 1] >> (16 * (e & 1)));
-                const uint16_t vh = (uint16_t)(vw[e >> 1] >> (16 * (e & 1)));
-                const float m_old = __half2float(__ushort_as_half(mh));
-                const float v_old = __half2float(__ushort_as_half(vh));
+                const float m_old = __half2float(__ushort_as_half((uint16_t)(mw[e >> 1] >> (16 * (e & 1)))));
+                const float v_old = __half2float(__ushort_as_half((uint16_t)(vw[e >> 1] >> (16 * (e & 1)))));
                 const float m1 = __fmaf_rn(b.beta1, m_old, __fmul_rn(b.omb1, gt));
                 const float v1 = __fmaf_rn(b.beta2, v_old, __fmul_rn(b.omb2, __fmul_rn(gt, gt)));
                 const float u = __fdiv_rn(__fmul_rn(m1, bc1),
@@ -177,50 +165,56 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
                     mout[e >> 1] = m16;
                     vout[e >> 1] = v16;
                 }
-                w[k][e] = Wn;
+                wn[e] = Wn;
                 amax = fmaxf(amax, fabsf(Wn));
             }
-            __stcs(reinterpret_cast<uint4 *>(d.m + grow + c0), make_uint4(mout[0], mout[1], mout[2], mout[3]));
-            __stcs(reinterpret_cast<uint4 *>(d.v + grow + c0), make_uint4(vout[0], vout[1], vout[2], vout[3]));
+            __stcs(reinterpret_cast<uint4 *>(mrow + c0), make_uint4(mout[0], mout[1], mout[2], mout[3]));
+            __stcs(reinterpret_cast<uint4 *>(vrow + c0), make_uint4(vout[0], vout[1], vout[2], vout[3]));
+            wrow4[2 * j] = make_float4(wn[0], wn[1], wn[2], wn[3]);
+            wrow4[2 * j + 1] = make_float4(wn[4], wn[5], wn[6], wn[7]);
         }
 
-        // new per-row scale from the row absmax (non-negative floats order as unsigned ints)
+        // new per-row scale from the row absmax (non-negative floats order as unsigned ints);
+        // the reduction's barriers also publish the shared-memory row to every thread
         const float rmax = __uint_as_float(block_max_u32(__float_as_uint(amax), max_scratch));
         const float sp = __fdiv_rn(rmax, 127.0f);
 
-#pragma unroll
-        for (int k = 0; k < CPT; ++k) {
-            const int j = tid + k * kThreads;
-            if (j >= nchunks) continue;
+        // ---- pass 2: requantise from shared memory, write q, delta and the live row ----
+        int8_t *qout = d.q + (size_t)r * C;
+        float *dout = d.delta + (size_t)r * C;
+        uint16_t *lout = d.live ? d.live + (size_t)r * C : nullptr;
+        for (int j = tid; j < nchunks; j += kThreads) {
             const int c0 = j << 3;
+            const float4 w0 = wrow4[2 * j], w1 = wrow4[2 * j + 1];
+            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
             uint32_t qo[2] = {0u, 0u};
             float dn[8];
             uint32_t lo16[4];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float Wn = w[k][e];
+                const float Wn = wv[e];
                 float qf = 0.0f, de = Wn;
                 if (sp != 0.0f) {
                     qf = rintf(__fdiv_rn(Wn, sp));
                     qf = fminf(fmaxf(qf, -127.0f), 127.0f);
                     de = __fmaf_rn(-sp, qf, Wn);
                 }
-                const int qi = (int)qf;
-                qo[e >> 2] |= ((uint32_t)qi & 0xFFu) << (8 * (e & 3));
+                qo[e >> 2] |= ((uint32_t)(int)qf & 0xFFu) << (8 * (e & 3));
                 dn[e] = de;
                 const uint16_t lb = __bfloat16_as_ushort(__float2bfloat16_rn(Wn));
                 if (e & 1) lo16[e >> 1] |= (uint32_t)lb << 16; else lo16[e >> 1] = lb;
             }
-            __stcs(reinterpret_cast<uint2 *>(d.q + wrow + c0), make_uint2(qo[0], qo[1]));
-            __stcs(reinterpret_cast<float4 *>(d.delta + wrow + c0), make_float4(dn[0], dn[1], dn[2], dn[3]));
-            __stcs(reinterpret_cast<float4 *>(d.delta + wrow + c0 + 4), make_float4(dn[4], dn[5], dn[6], dn[7]));
-            if (d.live)
-                __stcs(reinterpret_cast<uint4 *>(d.live + wrow + c0), make_uint4(lo16[0], lo16[1], lo16[2], lo16[3]));
+            __stcs(reinterpret_cast<uint2 *>(qout + c0), make_uint2(qo[0], qo[1]));
+            __stcs(reinterpret_cast<float4 *>(dout + c0), make_float4(dn[0], dn[1], dn[2], dn[3]));
+            __stcs(reinterpret_cast<float4 *>(dout + c0 + 4), make_float4(dn[4], dn[5], dn[6], dn[7]));
+            if (lout)
+                __stcs(reinterpret_cast<uint4 *>(lout + c0), make_uint4(lo16[0], lo16[1], lo16[2], lo16[3]));
         }
         if (tid == 0) {
             d.s[r] = sp;
             d.slot_step[slot] = t;
         }
+        __syncthreads();                 // the shared row is reused by the next item
     }
     if (nonfinite) set_status(status, SF_STATUS_NONFINITE);
 }
@@ -259,13 +253,6 @@ quantize_kernel(const float *W, int C, int8_t *q, float *s, float *delta, uint16
         if (live) live[row + c] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
     }
     if (threadIdx.x == 0) s[blockIdx.x] = sp;
-}
-
-template <int CPT>
-int launch_update(const UpdBatch &b, int grid, uint32_t *status, cudaStream_t st)
-{
-    update_kernel<CPT><<<grid, kThreads, 0, st>>>(b, status);
-    return launch_status();
 }
 
 }  // namespace
@@ -315,9 +302,16 @@ extern "C" int sf_sparse_update(const sf_matrix *mats, int n_mats, const sf_adam
         if (a.C > maxC) maxC = a.C;
     }
     if (n_mats == 0) return SF_OK;
-    const int cpt_needed = (maxC / 8 + kThreads - 1) / kThreads;
     const int sms = sm_count();
     if (sms <= 0) return SF_ERR_NO_DEVICE;
+    const size_t smem = (size_t)maxC * sizeof(float);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return SF_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, update_kernel, kThreads, smem) != cudaSuccess ||
+        per_sm <= 0)
+        return SF_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     for (int first = 0; first < n_mats; first += kMaxMatsPerLaunch) {
         const int cnt = n_mats - first < kMaxMatsPerLaunch ? n_mats - first : kMaxMatsPerLaunch;
@@ -355,17 +349,8 @@ extern "C" int sf_sparse_update(const sf_matrix *mats, int n_mats, const sf_adam
             d.pgrad = a.partner >= 0 ? mats[a.partner].grad : nullptr;
             d.prow_slot = a.partner >= 0 ? mats[a.partner].mask.row_slot : nullptr;
         }
-        const int grid = sms * 2;
-        int rc;
-        switch (cpt_needed) {
-        case 1: rc = launch_update<1>(b, grid, dev_status, st); break;
-        case 2: rc = launch_update<2>(b, grid, dev_status, st); break;
-        case 3: rc = launch_update<3>(b, grid, dev_status, st); break;
-        case 4: rc = launch_update<4>(b, grid, dev_status, st); break;
-        case 5: case 6: rc = launch_update<6>(b, grid, dev_status, st); break;
-        default: rc = launch_update<8>(b, grid, dev_status, st); break;
-        }
-        if (rc != SF_OK) return rc;
+        update_kernel<<<sms * per_sm, kThreads, smem, st>>>(b, dev_status);
+        if (launch_status() != SF_OK) return SF_ERR_CUDA;
     }
     return SF_OK;
 }

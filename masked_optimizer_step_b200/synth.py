@@ -178,3 +178,67 @@ def device_weights_f32(R: int, C: int, seed: int, *index: int, std: float = 0.02
     import torch
     gen = device_generator(seed, "weights", *index, device=device)
     return torch.randn((R, C), generator=gen, device=device, dtype=torch.float32).mul_(std)
+
+
+# ---------------------------------------------------------------------------------------------
+# The 7B-shaped step workload: per-projection chosen rows, one bank of step inputs, token stream.
+# ---------------------------------------------------------------------------------------------
+
+LAYER_INPUTS = ("x_attn", "attn_out", "x_ffn", "ffn_mid")
+
+
+def chosen_rows(seed: int, layer: int, idx: int, R: int, kind: str, bank: int) -> np.ndarray:
+    """Rows a projection's tracker should find active (~1%): `kind` is "scattered" (single
+    rows) or "clustered" (whole 32-row tiles). Bank 1 drifts ~5% of bank 0's choice."""
+    g = rng(seed, "rows", layer, idx)
+    rows = scattered_rows(g, R, 0.01) if kind == "scattered" else clustered_rows(g, R, 0.01)
+    if bank == 1:
+        g2 = rng(seed, "rows", layer, idx, 1)
+        if kind == "scattered":
+            k = max(1, int(round(0.05 * len(rows))))
+            keep = np.sort(g2.choice(len(rows), len(rows) - k, replace=False))
+            pool = np.setdiff1d(np.arange(R), rows)
+            rows = np.sort(np.concatenate([rows[keep], g2.choice(pool, k, replace=False)]))
+        else:
+            tiles = np.unique(rows // 32)
+            k = int(round(0.05 * len(tiles)))
+            if k:
+                pool = np.setdiff1d(np.arange(R // 32), tiles)
+                tiles = np.sort(np.concatenate([g2.choice(tiles, len(tiles) - k, replace=False),
+                                                g2.choice(pool, k, replace=False)]))
+                rows = (tiles[:, None] * 32 + np.arange(32)[None, :]).ravel()
+    return rows.astype(np.int64)
+
+
+def step_bank(projs, T: int, kind: str, bank: int, seed: int, hidden: int = 4096, device="cuda"):
+    """Device-resident inputs of one step for projections [(layer, name, R, C, input_name)]:
+    tracker outputs Y [T x R], output gradients dX [T x R], layer inputs A [T x C] (shared by the
+    projections that read the same input), and the embedding's upstream gradient dY [T x hidden]."""
+    import torch
+    Ys, dXs, As = [], [], []
+    inputs = {}
+    for i, (layer, name, R, C, inp) in enumerate(projs):
+        key = (layer, inp)
+        if key not in inputs:
+            inputs[key] = device_normal_bf16((T, C), seed, "act", bank, layer, LAYER_INPUTS.index(inp),
+                                             device=device)
+        As.append(inputs[key])
+        gain = torch.from_numpy(tracker_gains(R, chosen_rows(seed, layer, i, R, kind, bank))).to(device)
+        gen = device_generator(seed, "tracker", bank, i, device=device)
+        z = torch.randn((T, R), generator=gen, device=device, dtype=torch.float32)
+        Ys.append(z.mul_(gain[None, :]).to(torch.bfloat16))
+        del z
+        dXs.append(device_normal_bf16((T, R), seed, "dx", bank, i, device=device))
+    dY = device_normal_bf16((T, hidden), seed, "dy", bank, device=device)
+    return {"Y": Ys, "dX": dXs, "A": As, "dY": dY, "tokens": None, "distinct_A": list(inputs.values())}
+
+
+def token_stream(seed: int, n_windows: int, T: int, V: int = 32000, drift: float = 0.01) -> np.ndarray:
+    """n_windows batches of T token ids, Zipf(1.1) with a rank->id map drifting per window."""
+    g = rng(seed, "tokens")
+    rank_to_id = np.arange(V)
+    out = []
+    for _ in range(n_windows):
+        rank_to_id = drift_rank_map(g, rank_to_id, drift)
+        out.append(zipf_ids(g, T, V, 1.1, rank_to_id))
+    return np.stack(out)
