@@ -141,24 +141,60 @@ def token_stream(n_windows, T, V=32000):
 # algorithmic work per step, from the masks' counts
 # ---------------------------------------------------------------------------------------------
 
+def dw_groups(model):
+    """Consecutive projections reading the same layer input form one dW group (as the library
+    groups problems that share A)."""
+    from masked_optimizer_step_b200.model import INPUT_OF
+    groups = []
+    for i, p in enumerate(model.projs):
+        key = (p.layer, INPUT_OF[p.name])
+        if groups and groups[-1][0] == key and len(groups[-1][1]) < 8:
+            groups[-1][1].append(i)
+        else:
+            groups.append((key, [i]))
+    return [g for _, g in groups]
+
+
 def step_work(model, counts, T):
-    """counts: [n_mats, 8] host copy after a step. Returns dict of algorithmic work."""
+    """counts: [n_mats, 8] host copy after a step. Returns the step's algorithmic work.
+
+    Masked dW: per group, the device picks row mode when the group's active rows fit its scratch
+    (slot capacity rounded up to 32) and need fewer 128-row tiles than the mask tiles do; that
+    rule is mirrored here. Algorithmic bytes: A once per group, each active element of dX once
+    (row mode) or each active mask tile of dX once (tile mode), each dW row written once. FLOPs:
+    useful = 2*T*C per active row; executed = 2*T*C*128 per 128-row tile.
+    """
     off = 1 if model.emb is not None else 0
-    flops = 0
     upd_bytes = 0
     rows_updated = 0
     track_bytes = 0
     for i, m in enumerate(model.all_mats):
         c = counts[i]
-        rows, tiles, noslot, fresh = int(c[0]), int(c[1]), int(c[3]), int(c[4])
+        rows, noslot, fresh = int(c[0]), int(c[3]), int(c[4])
         upd_rows = rows - noslot
         rows_updated += upd_rows
         upd_bytes += (upd_rows - fresh) * m.C * 24 + fresh * m.C * 20 + upd_rows * 8
         if i >= off:
-            flops += 2 * T * m.C * 32 * tiles
             track_bytes += T * m.R * 2
+    dw_flops_exec = dw_flops_useful = dw_bytes = 0
+    rows_groups = 0
+    for grp in dw_groups(model):
+        mats = [model.projs[i].mat for i in grp]
+        cs = [counts[i + off] for i in grp]
+        rows = sum(int(c[0]) for c in cs)
+        tiles_mt = sum((int(c[1]) + 3) // 4 for c in cs)
+        mcap = -(-sum(m.mask.slot_cap for m in mats) // 32) * 32
+        rows_mode = rows <= mcap and -(-rows // 128) < tiles_mt
+        mt = -(-rows // 128) if rows_mode else tiles_mt
+        C = mats[0].C
+        dw_flops_exec += mt * 128 * C * T * 2
+        dw_flops_useful += rows * C * T * 2
+        dw_bytes += T * C * 2 + sum((int(c[0]) - int(c[3])) * C * 4 for c in cs)
+        dw_bytes += T * rows * 2 if rows_mode else sum(int(c[1]) * 32 * T * 2 for c in cs)
+        rows_groups += rows_mode
     emb = counts[0] if off else None
-    return {"dw_flops": flops, "update_bytes": upd_bytes, "rows_updated": rows_updated,
+    return {"dw_flops": dw_flops_exec, "dw_flops_useful": dw_flops_useful, "dw_bytes": dw_bytes,
+            "dw_row_groups": rows_groups, "update_bytes": upd_bytes, "rows_updated": rows_updated,
             "tracker_bytes": track_bytes, "active_rows": int(counts[:, 0].sum()),
             "active_tiles": int(counts[off:, 1].sum()), "emb_rows": int(emb[0]) if emb is not None else 0}
 
@@ -380,27 +416,48 @@ def main():
     hbm = float(peaks.get("hbm_gbs", 6650.0))
     tf_sus = float(peaks.get("bf16_tflops_sustained", 1400.0))
     dw_flops = sum(w["dw_flops"] for w in work)
+    dw_useful = sum(w["dw_flops_useful"] for w in work)
+    dw_bytes = sum(w["dw_bytes"] for w in work)
     upd_bytes = sum(w["update_bytes"] for w in work)
     trk_bytes = sum(w["tracker_bytes"] for w in work)
-    dw_tf = dw_flops / (stage_ms[1] / 1e3) / 1e12 if stage_ms[1] > 0 else 0.0
+    dw_s = stage_ms[1] / 1e3
+    dw_tf = dw_flops / dw_s / 1e12 if dw_s > 0 else 0.0
+    dw_gbs = dw_bytes / dw_s / 1e9 if dw_s > 0 else 0.0
     upd_gbs = upd_bytes / (stage_ms[3] / 1e3) / 1e9 if stage_ms[3] > 0 else 0.0
     trk_gbs = trk_bytes / (stage_ms[0] / 1e3) / 1e9 if stage_ms[0] > 0 else 0.0
+    # the dW roofline is whichever resource its algorithmic work needs longer on
+    dw_tensor_bound = dw_flops / (tf_sus * 1e12) >= dw_bytes / (hbm * 1e9)
+    dw_stage = {"ms_per_step": stage_ms[1] / args.steps,
+                "bound": "tensor" if dw_tensor_bound else "hbm",
+                "achieved": dw_tf if dw_tensor_bound else dw_gbs,
+                "peak": tf_sus if dw_tensor_bound else hbm,
+                "unit": "TFLOP/s" if dw_tensor_bound else "GB/s",
+                "frac": dw_tf / tf_sus if dw_tensor_bound else dw_gbs / hbm,
+                "tensor_tflops_executed": dw_tf, "tensor_frac_executed": dw_tf / tf_sus,
+                "tensor_tflops_useful": dw_useful / dw_s / 1e12 if dw_s > 0 else 0.0,
+                "hbm_gbs": dw_gbs, "hbm_frac": dw_gbs / hbm,
+                "row_mode_groups_per_step": work[-1]["dw_row_groups"],
+                "algorithmic": "bytes: A once per group + active dX once + dW rows; FLOP: 2*T*C per "
+                               "executed row (128-row tiles)"}
+    step_bytes = trk_bytes + dw_bytes + upd_bytes
     stages = {
         "masks": {"ms_per_step": stage_ms[0] / args.steps, "bound": "hbm", "achieved": trk_gbs,
                   "peak": hbm, "unit": "GB/s", "frac": trk_gbs / hbm, "algorithmic": "Y read once: T*R*2 B per projection"},
-        "masked_dw": {"ms_per_step": stage_ms[1] / args.steps, "bound": "tensor", "achieved": dw_tf,
-                      "peak": tf_sus, "unit": "TFLOP/s", "frac": dw_tf / tf_sus,
-                      "algorithmic": "2*T*C*32 FLOP per active 32-row tile"},
+        "masked_dw": dw_stage,
         "embed_grad": {"ms_per_step": stage_ms[2] / args.steps},
         "sparse_update": {"ms_per_step": stage_ms[3] / args.steps, "bound": "hbm", "achieved": upd_gbs,
                           "peak": hbm, "unit": "GB/s", "frac": upd_gbs / hbm,
                           "algorithmic": "24 B per active element (20 on fresh rows) + 8 B per row"},
     }
+    stages["step"] = {"hbm_floor_ms": step_bytes / args.steps / (hbm * 1e9) * 1e3,
+                      "frac_of_hbm_floor": (step_bytes / (hbm * 1e9)) / (ms_total / 1e3),
+                      "algorithmic_gb_per_step": step_bytes / args.steps / 1e9}
     dominant = max(("masks", "masked_dw", "sparse_update"), key=lambda s: stages[s]["ms_per_step"])
     d = stages[dominant]
     roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
                 "frac": d["frac"], "traffic": None, "kernel": dominant, "peak_source": peak_src,
-                "peak_kind": "sustained bf16 (kernel timed inside a long step)" if d["bound"] == "tensor" else "hbm copy"}
+                "peak_kind": "sustained bf16 (kernel timed inside a long step)" if d["bound"] == "tensor" else "hbm copy",
+                "algorithmic": d["algorithmic"]}
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -132,12 +132,19 @@ int sf_mask_update(const sf_mask *masks /* host [n_masks] */,
  * visited (nothing of it is loaded, multiplied or stored), and rows whose bit is clear inside
  * a live tile are discarded at the store. Active row r with slot k = row_slot[r] >= 0 gets
  *     dW[k * ld_dw + c] = sum_t dX[t, r] * A[t, c]      (fp32, accumulated in fp32 from bf16)
- * and nothing else of dW is written. Runs on the tensor cores (tcgen05, TMA) as one persistent
- * launch over the active tiles of all problems (up to SF_DW_MAX_PER_LAUNCH per launch).
- * Requirements: T >= 0; C a multiple of 8; ld_dx, ld_a multiples of 8; dX, A 16-byte aligned;
- * dW 16-byte aligned, ld_dw a multiple of 4 and >= C. Errors: SF_ERR_ARG, SF_ERR_ALIGN.
+ * and nothing else of dW is written. Runs on the tensor cores (tcgen05, TMA) as persistent
+ * launches over the work of all problems (as few launches as the kernel parameter space allows).
+ * Consecutive problems that read the same A (same pointer, ld_a, C and T: the q, k, v projections
+ * of a layer, or gate and up) are grouped: their rows share 128-row tensor-core tiles and A is
+ * streamed once per group. With scratch `ws` (sf_masked_dw_ws_bytes() bytes, 16-byte aligned)
+ * a group whose mask is scattered first gathers its active rows of dX into the scratch, so a
+ * tile holds 128 active rows instead of four 32-row mask tiles; the choice is made on the device
+ * from the live masks, per group, and does not change the result. With ws = NULL every group
+ * runs on mask tiles. Requirements: T >= 0; C a multiple of 8; when T > 0, ld_dx and ld_a
+ * multiples of 8 and dX, A 16-byte aligned; dW 16-byte aligned, ld_dw a multiple of 4 and >= C.
+ * Errors: SF_ERR_ARG (also for ws smaller than needed), SF_ERR_ALIGN.
  */
-#define SF_DW_MAX_PER_LAUNCH 64
+#define SF_DW_MAX_PER_LAUNCH 96   /* problems (and groups) per launch, at most */
 
 typedef struct sf_dw_problem {
     const void *dX;     /* bf16 [T x ld_dx] */
@@ -151,8 +158,10 @@ typedef struct sf_dw_problem {
     int64_t     ld_dw;
 } sf_dw_problem;
 
-int sf_masked_dw(const sf_dw_problem *probs /* host [n] */, int n, uint32_t *dev_status,
-                 sf_stream stream);
+size_t sf_masked_dw_ws_bytes(const sf_dw_problem *probs /* host [n] */, int n);
+
+int sf_masked_dw(const sf_dw_problem *probs /* host [n] */, int n, void *ws, size_t ws_bytes,
+                 uint32_t *dev_status, sf_stream stream);
 
 /* ---- sf_embed_grad: sections 1 and 2.2 (embedding rows) ---------------------------------
  * A row's gradient comes only from the batch positions holding its token, and only rows the

@@ -28,7 +28,9 @@ SF_SRC_OUTPUT_BF16 = 1
 SF_SRC_HITS_U32 = 2
 SF_SRC_WORDS = 3
 
-SF_DW_MAX_PER_LAUNCH = 64
+SF_DW_MAX_PER_LAUNCH = 96
+SF_MASKS_PER_LAUNCH = 240
+SF_MATS_PER_LAUNCH = 256
 
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -81,7 +83,9 @@ def load():
     L.sf_mask_init.argtypes = [ctypes.POINTER(sf_mask), _P]
     L.sf_mask_update.argtypes = [ctypes.POINTER(sf_mask), ctypes.POINTER(sf_mask_src), ctypes.c_int,
                                  _F, _P, _P]
-    L.sf_masked_dw.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int, _P, _P]
+    L.sf_masked_dw.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int, _P, ctypes.c_size_t, _P, _P]
+    L.sf_masked_dw_ws_bytes.restype = ctypes.c_size_t
+    L.sf_masked_dw_ws_bytes.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int]
     L.sf_embed_grad_ws_bytes.restype = ctypes.c_size_t
     L.sf_embed_grad_ws_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
     L.sf_embed_grad.argtypes = [_P, ctypes.c_int, _P, ctypes.c_int, _I64, ctypes.POINTER(sf_mask), _P,
@@ -216,11 +220,24 @@ def dw_problem(dX, A, mask: Mask, dW) -> Desc:
     return Desc(c, dX, A, dW)
 
 
-def sf_masked_dw(problems, status=None, stream=None):
-    """problems: list of dw_problem() descriptors."""
+def sf_masked_dw_ws_bytes(problems) -> int:
     n = len(problems)
     arr = (sf_dw_problem * n)(*[p.c for p in problems])
-    _check(load().sf_masked_dw(arr, n, _ptr(status), _stream(stream)), "sf_masked_dw")
+    return load().sf_masked_dw_ws_bytes(arr, n)
+
+
+def dw_workspace(problems, device="cuda") -> torch.Tensor:
+    """Scratch for sf_masked_dw's row mode (a byte tensor of sf_masked_dw_ws_bytes bytes)."""
+    return torch.empty(max(sf_masked_dw_ws_bytes(problems), 1), dtype=torch.uint8, device=device)
+
+
+def sf_masked_dw(problems, status=None, stream=None, ws=None):
+    """problems: list of dw_problem() descriptors; ws: dw_workspace() scratch, or None for the
+    mask-tile mode only."""
+    n = len(problems)
+    arr = (sf_dw_problem * n)(*[p.c for p in problems])
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(load().sf_masked_dw(arr, n, _ptr(ws), nbytes, _ptr(status), _stream(stream)), "sf_masked_dw")
 
 
 def sf_embed_grad_ws_bytes(n_tok: int, slot_cap: int) -> int:

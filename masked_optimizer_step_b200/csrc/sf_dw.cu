@@ -9,61 +9,91 @@
 // GEMM terms M = weight rows, N = columns, K = tokens, and BOTH operands are M/N-contiguous
 // ("MN-major"): tcgen05 reads them that way directly, so nothing is transposed in memory.
 //
-// Work: the mask's ascending active-tile list is cut into M-tiles of four 32-row tiles (128
-// rows, gathered from anywhere in the matrix); each M-tile x 256-column N-tile is one unit.
-// All-empty tiles never appear in the list, so they cost nothing at all. One persistent launch
-// walks the units of every projection of the call (problem-major, so a projection's A stays in
-// L2 while its units run).
+// Groups. Consecutive problems of a call that read the same A (same pointer, stride, C and T --
+// e.g. the q, k and v projections of a layer, or gate and up) form a group: their rows share
+// M-tiles and A is streamed once per group. Each group runs in one of two modes, chosen on the
+// device from the live masks (no host readback):
+//   tile mode  the pages' design: the ascending list of active 32-row tiles of each problem is
+//              cut into 128-row M-tiles of four tiles, gathered straight from dX by TMA; rows of
+//              a live tile that are inactive are computed and dropped at the store.
+//   row mode   a gather kernel first copies just the active rows of every problem of the group
+//              into a dense token-major buffer (caller scratch), so an M-tile holds 128 active
+//              rows instead of four tiles. Same result; far fewer tensor-core FLOPs when rows are
+//              scattered (at 1% scattered rows, a live tile holds ~1.2 active rows).
+// Row mode is used when the group's active rows fit the scratch and it needs fewer M-tiles.
 //
-// CTA (1 per SM, 192 threads, warp-specialised):
-//   warp 0      TMA producer: per 64-token stage, four 32-row boxes of dX (SWIZZLE_64B) and
-//               four 64-column boxes of A (SWIZZLE_128B) into a 4-deep shared-memory ring;
+// CTA (1 per SM, 192 threads, warp-specialised, persistent over the units of the launch):
+//   warp 0      TMA producer: per 64-token stage, four 32-row boxes of the A-operand
+//               (SWIZZLE_64B) and four 64-column boxes of A (SWIZZLE_128B) into a 4-deep ring;
 //   warp 1      allocates 512 TMEM columns, one thread issues tcgen05.mma kind::f16
 //               (M=128, N=256, K=16, bf16 in, fp32 accumulate) into one of two 256-column
-//               accumulators, and commits stage releases / accumulator-ready to mbarriers;
+//               accumulators and commits stage releases / accumulator-ready to mbarriers;
 //   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns at a time (warp w reads TMEM lanes
-//               32*(w%4)..), tests each row's mask bit and slot, stores fp32 rows of dW.
-// The two accumulators let the epilogue of one unit overlap the main loop of the next.
+//               32*(w%4)..), maps each lane to its weight row and slot, stores fp32 rows of dW.
 // Every mbarrier wait is bounded (2 s): on expiry the CTA raises SF_STATUS_WAIT_TIMEOUT, drains
 // its own TMA loads, frees its TMEM and exits.
+#include <string.h>
+
 #include "sf_common.cuh"
 #include "sf_host.h"
 
 namespace sf {
 namespace {
 
-constexpr int BM = 128;                 // rows per unit: four 32-row mask tiles
+constexpr int BM = 128;                 // rows per unit
 constexpr int BN = 256;                 // columns per unit
 constexpr int BK = 64;                  // tokens per pipeline stage
 constexpr int UMMA_K = 16;              // K of one tcgen05.mma kind::f16
 constexpr int STAGES = 4;
-constexpr int A_TILE_BYTES = 32 * BK * 2;          // one 32-row tile x 64 tokens (64 B rows)
+constexpr int A_TILE_BYTES = 32 * BK * 2;          // 32 rows x 64 tokens (64 B rows)
 constexpr int A_STAGE_BYTES = 4 * A_TILE_BYTES;    // 16 KB
 constexpr int B_BOX_BYTES = 64 * BK * 2;           // 64 columns x 64 tokens (128 B rows)
 constexpr int B_STAGE_BYTES = (BN / 64) * B_BOX_BYTES;   // 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int kThreads = 192;
-constexpr int kMaxProblems = SF_DW_MAX_PER_LAUNCH;
 constexpr size_t kSmemBytes = (size_t)STAGES * STAGE_BYTES + 1024;   // + alignment slack
+constexpr int kMaxPerGroup = 8;
+constexpr int kInfoInts = 16;           // per group: mode, total rows, row prefix [kMaxPerGroup+1]
+constexpr int kGatherTokens = 32;       // tokens per gather CTA
+constexpr int kGatherThreads = 256;
 
-struct alignas(64) DwDesc {
-    CUtensorMap tm_dx;           // dims {R, T}, box {32, 64}, 64-byte swizzle
-    CUtensorMap tm_a;            // dims {C, T}, box {64, 64}, 128-byte swizzle
-    const uint32_t *words;
+struct alignas(64) DwProb {
+    CUtensorMap tm_dx;           // dX: dims {R, T}, box {32, 64}, 64-byte swizzle
+    const uint16_t *dx;
     const int32_t *active_tiles;
+    const int32_t *active_rows;
     const int32_t *counts;
     const int32_t *row_slot;
     float *dW;
-    int64_t ld_dw;
-    int32_t R, C, T, n_ntiles;
+    int32_t ld_dx, ld_dw, R, group;
 };
 
-struct DwBatch {
-    int32_t n;
-    DwDesc d[kMaxProblems];
+struct alignas(64) DwGroup {
+    CUtensorMap tm_a;            // A: dims {C, T}, box {64, 64}, 128-byte swizzle
+    CUtensorMap tm_g;            // gathered rows: dims {mcap, T}, box {32, 64}, 64-byte swizzle
+    uint16_t *dxg;               // gathered rows, T x mcap bf16 (null: tile mode only)
+    int32_t *info;               // device: [0] mode (1 = rows), [1] rows, [2..] row prefix
+    int32_t first, count, C, T, n_ntiles, mcap;
 };
-static_assert(sizeof(DwBatch) < 32000, "kernel parameter space");
+
+constexpr int kParamBudget = 32764;
+
+struct DwBatch {
+    int32_t n_prob, n_group;
+    // variable-length payload: n_group DwGroup then n_prob DwProb
+    alignas(64) unsigned char payload[32640];
+};
+static_assert(sizeof(DwBatch) <= kParamBudget, "kernel parameter space");
+
+__device__ __forceinline__ const DwGroup &grp(const DwBatch &b, int g)
+{
+    return reinterpret_cast<const DwGroup *>(b.payload)[g];
+}
+__device__ __forceinline__ const DwProb &prb(const DwBatch &b, int p)
+{
+    return reinterpret_cast<const DwProb *>(b.payload + (size_t)b.n_group * sizeof(DwGroup))[p];
+}
 
 // Shared-memory matrix descriptor (tcgen05 "matrix descriptor"): start address, leading and
 // stride byte offsets (16-byte units), version 1, swizzle mode in bits 61..63.
@@ -82,24 +112,120 @@ constexpr uint32_t kLayoutSW64 = 4;
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                             ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-struct Unit {
-    int p, mt, nt;
+// Mode and size of a group, from the live masks. Every reader computes the same answer.
+struct GroupPlan {
+    int rows_mode;      // 1: row mode
+    int m_tiles;        // M-tiles of the group in its mode
+    int total_rows;     // active rows of all problems of the group
 };
 
-__device__ __forceinline__ Unit decode(int u, const int *prefix, int n, const DwBatch &b)
+__device__ __forceinline__ GroupPlan plan_group(const DwBatch &b, const DwGroup &g)
 {
-    int lo = 0, hi = n - 1;
+    int rows = 0, tiles_mt = 0;
+    for (int k = 0; k < g.count; ++k) {
+        const DwProb &p = prb(b, g.first + k);
+        rows += p.counts[0];
+        tiles_mt += (p.counts[1] + 3) >> 2;
+    }
+    const int rows_mt = (rows + BM - 1) / BM;
+    GroupPlan pl;
+    pl.rows_mode = g.dxg != nullptr && rows <= g.mcap && rows_mt < tiles_mt;
+    pl.m_tiles = pl.rows_mode ? rows_mt : tiles_mt;
+    pl.total_rows = rows;
+    return pl;
+}
+
+// ------------------------------------ gather kernel ------------------------------------
+// Row mode only: dxg[t, k] = dX_p[t, active_rows_p[k - prefix_p]] for the group's k-th active
+// row. One CTA per (group, 32 tokens); the first CTA of a group also records the plan, which the
+// main kernel (next on the stream) reads.
+__global__ void __launch_bounds__(kGatherThreads)
+dw_gather_kernel(const __grid_constant__ DwBatch b, int blocks_per_group)
+{
+    const int gi = blockIdx.x / blocks_per_group;
+    const int tb = blockIdx.x - gi * blocks_per_group;
+    const DwGroup &g = grp(b, gi);
+    if (g.dxg == nullptr) return;
+    const GroupPlan pl = plan_group(b, g);
+    __shared__ int prefix[kMaxPerGroup + 1];
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int k = 0; k < g.count; ++k) {
+            prefix[k] = acc;
+            acc += prb(b, g.first + k).counts[0];
+        }
+        prefix[g.count] = acc;
+        if (tb == 0) {
+            g.info[0] = pl.rows_mode;
+            g.info[1] = acc;
+            for (int k = 0; k <= g.count; ++k) g.info[2 + k] = prefix[k];
+        }
+    }
+    __syncthreads();
+    if (!pl.rows_mode) return;
+    const int t0 = tb * kGatherTokens;
+    const int nt = min(g.T - t0, kGatherTokens);
+    if (nt <= 0) return;
+    for (int k = threadIdx.x; k < pl.total_rows; k += kGatherThreads) {
+        int p = 0;
+        while (p + 1 < g.count && prefix[p + 1] <= k) ++p;
+        const DwProb &pr = prb(b, g.first + p);
+        const int r = pr.active_rows[k - prefix[p]];
+        const uint16_t *src = pr.dx + (size_t)t0 * pr.ld_dx + r;
+        uint16_t *dst = g.dxg + (size_t)t0 * g.mcap + k;
+        uint16_t v[kGatherTokens];
+#pragma unroll
+        for (int j = 0; j < kGatherTokens; ++j)
+            if (j < nt) v[j] = __ldcs(src + (size_t)j * pr.ld_dx);
+#pragma unroll
+        for (int j = 0; j < kGatherTokens; ++j)
+            if (j < nt) dst[(size_t)j * g.mcap] = v[j];
+    }
+}
+
+// ------------------------------------ unit decoding ------------------------------------
+
+struct Unit {
+    int g;          // group
+    int mt;         // M-tile within the group (row mode) or within problem p (tile mode)
+    int nt;         // N-tile
+    int p;          // problem (tile mode), -1 in row mode
+    int rows_mode;
+};
+
+struct SmemPlan {
+    int unit_prefix[SF_DW_MAX_PER_LAUNCH + 1];     // per group
+    int rows_mode[SF_DW_MAX_PER_LAUNCH];
+    int mt_prefix[SF_DW_MAX_PER_LAUNCH + 1];       // per problem: M-tiles before it in its group
+};
+
+__device__ __forceinline__ Unit decode(int u, const SmemPlan &sp, const DwBatch &b)
+{
+    int lo = 0, hi = b.n_group - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (prefix[mid] <= u) lo = mid; else hi = mid - 1;
+        if (sp.unit_prefix[mid] <= u) lo = mid; else hi = mid - 1;
     }
-    const int local = u - prefix[lo];
+    const DwGroup &g = grp(b, lo);
+    const int local = u - sp.unit_prefix[lo];
     Unit x;
-    x.p = lo;
-    x.mt = local / b.d[lo].n_ntiles;
-    x.nt = local - x.mt * b.d[lo].n_ntiles;
+    x.g = lo;
+    x.rows_mode = sp.rows_mode[lo];
+    const int mt = local / g.n_ntiles;
+    x.nt = local - mt * g.n_ntiles;
+    if (x.rows_mode) {
+        x.mt = mt;
+        x.p = -1;
+    } else {
+        int p = g.first;
+        while (p + 1 < g.first + g.count && sp.mt_prefix[p + 1] <= mt) ++p;
+        x.p = p;
+        x.mt = mt - sp.mt_prefix[p];
+    }
     return x;
 }
+
+// ------------------------------------ main kernel ------------------------------------
 
 __global__ void __launch_bounds__(kThreads, 1)
 masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
@@ -107,20 +233,30 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2], tempty_bar[2], drain_bar;
     __shared__ uint32_t tmem_base_s;
-    __shared__ int prefix[kMaxProblems + 1];
+    __shared__ SmemPlan sp;
     __shared__ int scan_scratch[33];
     __shared__ volatile int abort_flag;
 
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    {   // units per problem: ceil(active tiles / 4) M-tiles x N-tiles
+    {   // per group: mode and units; per problem: M-tiles before it inside its group
         int units = 0;
-        if (tid < b.n) units = ((b.d[tid].counts[1] + 3) >> 2) * b.d[tid].n_ntiles;
+        if (tid < b.n_group) {
+            const DwGroup &g = grp(b, tid);
+            const GroupPlan pl = plan_group(b, g);
+            sp.rows_mode[tid] = pl.rows_mode;
+            units = pl.m_tiles * g.n_ntiles;
+            int acc = 0;
+            for (int k = 0; k < g.count; ++k) {
+                sp.mt_prefix[g.first + k] = acc;
+                acc += (prb(b, g.first + k).counts[1] + 3) >> 2;
+            }
+        }
         int total;
         const int off = block_exclusive_scan(units, scan_scratch, &total);
-        if (tid < b.n) prefix[tid] = off;
-        if (tid == 0) prefix[b.n] = total;
+        if (tid < b.n_group) sp.unit_prefix[tid] = off;
+        if (tid == 0) sp.unit_prefix[b.n_group] = total;
     }
     if (tid == 0) {
         abort_flag = 0;
@@ -140,14 +276,14 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_s;
-    const int total_units = prefix[b.n];
+    const int total_units = sp.unit_prefix[b.n_group];
 
     if (warp == 0) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
-            for (int i = 0; i < b.n; ++i) {
-                prefetch_tmap(&b.d[i].tm_dx);
-                prefetch_tmap(&b.d[i].tm_a);
+            for (int i = 0; i < b.n_group; ++i) {
+                prefetch_tmap(&grp(b, i).tm_a);
+                if (sp.rows_mode[i]) prefetch_tmap(&grp(b, i).tm_g);
             }
             int stage = 0;
             uint32_t phase = 0;
@@ -155,17 +291,31 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             uint32_t issued_parity[STAGES] = {0, 0, 0, 0};
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-                const Unit x = decode(u, prefix, b.n, b);
-                const DwDesc &d = b.d[x.p];
-                const int nk = (d.T + BK - 1) / BK;
-                const int n_tiles = d.counts[1];
-                int tile[4];
+                const Unit x = decode(u, sp, b);
+                const DwGroup &g = grp(b, x.g);
+                const int nk = (g.T + BK - 1) / BK;
+                const CUtensorMap *tm_rows;
+                int coord[4];
                 int nvalid = 0;
+                if (x.rows_mode) {
+                    tm_rows = &g.tm_g;
+                    const int total = g.info[1];
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
-                    const int idx = x.mt * 4 + s;
-                    tile[s] = idx < n_tiles ? d.active_tiles[idx] : -1;
-                    nvalid += tile[s] >= 0;
+                    for (int s = 0; s < 4; ++s) {
+                        const int k0 = x.mt * BM + s * 32;
+                        coord[s] = k0 < total ? k0 : -1;
+                        nvalid += coord[s] >= 0;
+                    }
+                } else {
+                    const DwProb &p = prb(b, x.p);
+                    tm_rows = &p.tm_dx;
+                    const int n_tiles = p.counts[1];
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        const int idx = x.mt * 4 + s;
+                        coord[s] = idx < n_tiles ? p.active_tiles[idx] * 32 : -1;
+                        nvalid += coord[s] >= 0;
+                    }
                 }
                 const uint32_t bytes = nvalid * A_TILE_BYTES + B_STAGE_BYTES;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -175,11 +325,11 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     mbar_arrive_expect_tx(&full_bar[stage], bytes);
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
-                        if (tile[s] >= 0)
-                            tma_load_2d(sa + s * A_TILE_BYTES, &d.tm_dx, &full_bar[stage], tile[s] * 32, kb * BK);
+                        if (coord[s] >= 0)
+                            tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
 #pragma unroll
                     for (int j = 0; j < BN / 64; ++j)
-                        tma_load_2d(sb + j * B_BOX_BYTES, &d.tm_a, &full_bar[stage], x.nt * BN + j * 64, kb * BK);
+                        tma_load_2d(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], x.nt * BN + j * 64, kb * BK);
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -204,8 +354,8 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             uint32_t acc_phase = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-                const Unit x = decode(u, prefix, b.n, b);
-                const int nk = (b.d[x.p].T + BK - 1) / BK;
+                const Unit x = decode(u, sp, b);
+                const int nk = (grp(b, x.g).T + BK - 1) / BK;
                 if (nk == 0) continue;
                 if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -217,7 +367,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     const uint32_t sb = sa + A_STAGE_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
-                        // 16 tokens = 16 rows of 64 B (A) or 128 B (B)
+                        // 16 tokens = 16 rows of 64 B (A-operand) or 128 B (B-operand)
                         const uint64_t da = smem_desc(sa + k * UMMA_K * 64, A_TILE_BYTES, 8 * 64, kLayoutSW64);
                         const uint64_t db = smem_desc(sb + k * UMMA_K * 128, B_BOX_BYTES, 8 * 128, kLayoutSW128);
                         mma_bf16(d_tmem, da, db, kIdesc, (kb | k) != 0);
@@ -240,20 +390,30 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-            const Unit x = decode(u, prefix, b.n, b);
-            const DwDesc &d = b.d[x.p];
-            const int nk = (d.T + BK - 1) / BK;
-            const int idx = x.mt * 4 + quad;
+            const Unit x = decode(u, sp, b);
+            const DwGroup &g = grp(b, x.g);
+            const int nk = (g.T + BK - 1) / BK;
+            // the weight row of this lane's accumulator row, its slot and its output
             int slot = -1;
-            if (idx < d.counts[1]) {
-                const int tile = d.active_tiles[idx];
-                if ((d.words[tile] >> lane) & 1u) slot = d.row_slot[tile * 32 + lane];
+            const DwProb *p = nullptr;
+            if (x.rows_mode) {
+                const int k = x.mt * BM + quad * 32 + lane;
+                if (k < g.info[1]) {
+                    int q = 0;
+                    while (q + 1 < g.count && g.info[2 + q + 1] <= k) ++q;
+                    p = &prb(b, g.first + q);
+                    slot = p->row_slot[p->active_rows[k - g.info[2 + q]]];
+                }
+            } else {
+                p = &prb(b, x.p);
+                const int idx = x.mt * 4 + quad;
+                if (idx < p->counts[1]) slot = p->row_slot[p->active_tiles[idx] * 32 + lane];
             }
             const int col_base = x.nt * BN;
-            float *out = slot >= 0 ? d.dW + (size_t)slot * d.ld_dw : nullptr;
+            float *out = slot >= 0 ? p->dW + (size_t)slot * p->ld_dw : nullptr;
             if (nk == 0) {                      // no tokens: the gradient is zero
                 if (out)
-                    for (int c = col_base; c < min(d.C, col_base + BN); c += 4)
+                    for (int c = col_base; c < min(g.C, col_base + BN); c += 4)
                         *reinterpret_cast<float4 *>(out + c) = make_float4(0.f, 0.f, 0.f, 0.f);
                 continue;
             }
@@ -268,10 +428,10 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 tmem_ld_32x32b_x32(t_row + cc * 32, v);
                 tmem_ld_wait();
                 const int c0 = col_base + cc * 32;
-                if (out && c0 < d.C) {
+                if (out && c0 < g.C) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        if (c0 + 4 * j < d.C)
+                        if (c0 + 4 * j < g.C)
                             *reinterpret_cast<float4 *>(out + c0 + 4 * j) =
                                 make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
@@ -315,7 +475,7 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// bf16 2-D map over a token-major matrix [rows_T x ld], `width` valid columns, box {bx, 64}.
+// bf16 2-D map over a token-major matrix [T x ld], `width` valid columns, box {bx, 64}.
 bool encode_bf16(CUtensorMap *m, const void *base, int width, int T, int64_t ld, int bx,
                  CUtensorMapSwizzle sw)
 {
@@ -330,12 +490,59 @@ bool encode_bf16(CUtensorMap *m, const void *base, int width, int T, int64_t ld,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Groups of a call: runs of consecutive problems with the same A, stride, C and T.
+struct HostGroup {
+    int first, count;
+    int mcap;                    // gathered-row capacity (multiple of 32)
+    size_t ws_off;               // byte offset of the group's scratch (info block, then rows)
+};
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr size_t kInfoBytes = 256;      // info block, padded so the rows start 256-aligned
+
+int plan_groups(const sf_dw_problem *probs, int n, HostGroup *out, size_t *ws_total)
+{
+    int ng = 0;
+    size_t off = 0;
+    for (int i = 0; i < n;) {
+        int j = i + 1;
+        while (j < n && j - i < kMaxPerGroup && probs[j].A == probs[i].A && probs[j].ld_a == probs[i].ld_a &&
+               probs[j].C == probs[i].C && probs[j].T == probs[i].T)
+            ++j;
+        HostGroup &g = out[ng++];
+        g.first = i;
+        g.count = j - i;
+        size_t cap = 0;
+        for (int k = i; k < j; ++k) cap += (size_t)probs[k].mask.slot_cap;
+        g.mcap = (int)round_up(cap, 32);
+        g.ws_off = off;
+        off += kInfoBytes + round_up((size_t)(probs[i].T > 0 ? probs[i].T : 0) * g.mcap * 2, 256);
+        i = j;
+    }
+    *ws_total = off;
+    return ng;
+}
+
+size_t launch_bytes(const HostGroup &g) { return sizeof(DwGroup) + (size_t)g.count * sizeof(DwProb); }
+
 }  // namespace
 }  // namespace sf
 
 using namespace sf;
 
-extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, uint32_t *dev_status, sf_stream stream)
+extern "C" size_t sf_masked_dw_ws_bytes(const sf_dw_problem *probs, int n)
+{
+    if (n <= 0 || !probs) return 0;
+    HostGroup *groups = new HostGroup[n];
+    size_t total = 0;
+    plan_groups(probs, n, groups, &total);
+    delete[] groups;
+    return total;
+}
+
+extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t ws_bytes,
+                            uint32_t *dev_status, sf_stream stream)
 {
     if (n < 0 || (n > 0 && !probs)) return SF_ERR_ARG;
     for (int i = 0; i < n; ++i) {
@@ -343,51 +550,115 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, uint32_t *dev_sta
         int rc = check_mask(p.mask);
         if (rc != SF_OK) return rc;
         if (p.T < 0 || p.C <= 0 || (p.C & 7) || !p.dW) return SF_ERR_ARG;
-        if (p.ld_dw < p.C) return SF_ERR_ARG;
+        if (p.ld_dw < p.C || p.ld_dw > INT32_MAX) return SF_ERR_ARG;
         if ((p.ld_dw & 3) || !aligned16(p.dW)) return SF_ERR_ALIGN;
         if (p.T > 0) {                       // dX and A are read only when there are tokens
-            if (!p.dX || !p.A || p.ld_dx < p.mask.R || p.ld_a < p.C) return SF_ERR_ARG;
+            if (!p.dX || !p.A || p.ld_dx < p.mask.R || p.ld_a < p.C || p.ld_dx > INT32_MAX) return SF_ERR_ARG;
             if ((p.ld_dx & 7) || (p.ld_a & 7) || !aligned16(p.dX) || !aligned16(p.A)) return SF_ERR_ALIGN;
         }
     }
     if (n == 0) return SF_OK;
-    const int sms = sm_count();
-    if (sms <= 0) return SF_ERR_NO_DEVICE;
+    HostGroup *groups = new HostGroup[n];
+    size_t need = 0;
+    const int ng = plan_groups(probs, n, groups, &need);
+    const bool use_ws = ws != nullptr;
+    int rc = SF_OK;
+    if (use_ws && ws_bytes < need) rc = SF_ERR_ARG;
+    else if (use_ws && !aligned16(ws)) rc = SF_ERR_ALIGN;
+    const int sms = rc == SF_OK ? sm_count() : 0;
+    if (rc == SF_OK && sms <= 0) rc = SF_ERR_NO_DEVICE;
+    if (rc == SF_OK && cudaFuncSetAttribute(masked_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            (int)kSmemBytes) != cudaSuccess)
+        rc = SF_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
-    if (cudaFuncSetAttribute(masked_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemBytes) != cudaSuccess)
-        return SF_ERR_CUDA;
-    for (int first = 0; first < n; first += kMaxProblems) {
-        const int cnt = n - first < kMaxProblems ? n - first : kMaxProblems;
-        DwBatch batch;
-        memset(&batch, 0, sizeof(batch));
-        batch.n = cnt;
+    // Split the groups over as few launches as the parameter space allows, evenly by size.
+    const size_t payload = sizeof(DwBatch::payload);
+    size_t all = 0;
+    for (int k = 0; k < ng; ++k) all += launch_bytes(groups[k]);
+    int n_launch = (int)((all + payload - 1) / payload);
+    DwBatch *batch = rc == SF_OK ? new DwBatch : nullptr;
+    int gi = 0;
+    for (int li = 0; rc == SF_OK && gi < ng; ++li) {
+        size_t left = 0;
+        for (int k = gi; k < ng; ++k) left += launch_bytes(groups[k]);
+        const int launches_left = n_launch - li > 1 ? n_launch - li : 1;
+        const size_t target = (left + launches_left - 1) / launches_left;
+        int g_end = gi, np = 0;
+        size_t used = 0;
+        while (g_end < ng) {
+            const size_t add = launch_bytes(groups[g_end]);
+            if (g_end > gi && (used + add > payload || used >= target)) break;
+            if (g_end - gi + 1 > SF_DW_MAX_PER_LAUNCH || np + groups[g_end].count > SF_DW_MAX_PER_LAUNCH) break;
+            used += add;
+            np += groups[g_end].count;
+            ++g_end;
+        }
+        if (g_end == gi) { rc = SF_ERR_UNSUPPORTED; break; }
+        if (g_end < ng && li + 1 >= n_launch) ++n_launch;     // an uneven split needs one more
+        memset(batch, 0, sizeof(*batch));
+        batch->n_group = g_end - gi;
+        batch->n_prob = np;
+        DwGroup *gd = reinterpret_cast<DwGroup *>(batch->payload);
+        DwProb *pd = reinterpret_cast<DwProb *>(batch->payload + (size_t)batch->n_group * sizeof(DwGroup));
         long long max_units = 0;
-        for (int j = 0; j < cnt; ++j) {
-            const sf_dw_problem &p = probs[first + j];
-            DwDesc &d = batch.d[j];
-            const void *dx = p.T > 0 ? p.dX : p.dW;     // any valid address when there are no tokens
-            const void *a = p.T > 0 ? p.A : p.dW;
-            if (!encode_bf16(&d.tm_dx, dx, p.mask.R, p.T, p.T > 0 ? p.ld_dx : p.mask.R, 32,
-                             CU_TENSOR_MAP_SWIZZLE_64B) ||
-                !encode_bf16(&d.tm_a, a, p.C, p.T, p.T > 0 ? p.ld_a : p.C, 64,
-                             CU_TENSOR_MAP_SWIZZLE_128B))
-                return SF_ERR_CUDA;
-            d.words = p.mask.words;
-            d.active_tiles = p.mask.active_tiles;
-            d.counts = p.mask.counts;
-            d.row_slot = p.mask.row_slot;
-            d.dW = p.dW;
-            d.ld_dw = p.ld_dw;
-            d.R = p.mask.R;
-            d.C = p.C;
-            d.T = p.T;
-            d.n_ntiles = (p.C + BN - 1) / BN;
-            max_units += (long long)((p.mask.R / 32 + 3) / 4) * d.n_ntiles;
+        int pi = 0;
+        int tok_blocks = 1;
+        for (int k = gi; k < g_end && rc == SF_OK; ++k) {
+            const HostGroup &hg = groups[k];
+            const sf_dw_problem &p0 = probs[hg.first];
+            DwGroup &g = gd[k - gi];
+            const void *a = p0.T > 0 ? p0.A : p0.dW;     // any valid address when there are no tokens
+            if (!encode_bf16(&g.tm_a, a, p0.C, p0.T, p0.T > 0 ? p0.ld_a : p0.C, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+                rc = SF_ERR_CUDA;
+            g.first = pi;
+            g.count = hg.count;
+            g.C = p0.C;
+            g.T = p0.T;
+            g.n_ntiles = (p0.C + BN - 1) / BN;
+            g.mcap = hg.mcap;
+            if (use_ws && p0.T > 0 && hg.mcap > 0) {
+                uint8_t *base = static_cast<uint8_t *>(ws) + hg.ws_off;
+                g.info = reinterpret_cast<int32_t *>(base);
+                g.dxg = reinterpret_cast<uint16_t *>(base + kInfoBytes);
+                if (!encode_bf16(&g.tm_g, g.dxg, hg.mcap, p0.T, hg.mcap, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+                    rc = SF_ERR_CUDA;
+                tok_blocks = max(tok_blocks, (p0.T + kGatherTokens - 1) / kGatherTokens);
+            }
+            long long tiles_mt = 0;
+            for (int q = 0; q < hg.count; ++q, ++pi) {
+                const sf_dw_problem &p = probs[hg.first + q];
+                DwProb &d = pd[pi];
+                const void *dx = p.T > 0 ? p.dX : p.dW;
+                if (!encode_bf16(&d.tm_dx, dx, p.mask.R, p.T, p.T > 0 ? p.ld_dx : p.mask.R, 32,
+                                 CU_TENSOR_MAP_SWIZZLE_64B))
+                    rc = SF_ERR_CUDA;
+                d.dx = static_cast<const uint16_t *>(p.dX);
+                d.active_tiles = p.mask.active_tiles;
+                d.active_rows = p.mask.active_rows;
+                d.counts = p.mask.counts;
+                d.row_slot = p.mask.row_slot;
+                d.dW = p.dW;
+                d.ld_dx = (int32_t)p.ld_dx;
+                d.ld_dw = (int32_t)p.ld_dw;
+                d.R = p.mask.R;
+                d.group = k - gi;
+                tiles_mt += (p.mask.R / 32 + 3) / 4;
+            }
+            max_units += tiles_mt * g.n_ntiles;
+        }
+        if (rc != SF_OK) break;
+        if (use_ws) {
+            dw_gather_kernel<<<batch->n_group * tok_blocks, kGatherThreads, 0, st>>>(*batch, tok_blocks);
+            if (launch_status() != SF_OK) { rc = SF_ERR_CUDA; break; }
         }
         const int grid = (int)(max_units < sms ? max_units : sms);
-        masked_dw_kernel<<<grid, kThreads, kSmemBytes, st>>>(batch, dev_status);
-        if (launch_status() != SF_OK) return SF_ERR_CUDA;
+        if (grid > 0) {
+            masked_dw_kernel<<<grid, kThreads, kSmemBytes, st>>>(*batch, dev_status);
+            if (launch_status() != SF_OK) { rc = SF_ERR_CUDA; break; }
+        }
+        gi = g_end;
     }
-    return SF_OK;
+    delete batch;
+    delete[] groups;
+    return rc;
 }

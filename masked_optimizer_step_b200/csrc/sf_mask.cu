@@ -47,14 +47,14 @@ struct MaskDesc {
     int32_t tok_segs;     // OUTPUT: token segments
 };
 
-constexpr int kMaxMasksPerLaunch = 200;
+constexpr int kMaxMasksPerLaunch = 240;
 
 struct MaskBatch {
     int32_t n;
     int32_t total_ctas;
     MaskDesc d[kMaxMasksPerLaunch];
 };
-static_assert(sizeof(MaskBatch) < 32000, "kernel parameter space");
+static_assert(sizeof(MaskBatch) <= 32764, "kernel parameter space");
 
 __device__ __forceinline__ int find_mask(const MaskBatch &b, int cta)
 {

@@ -26,7 +26,7 @@ namespace sf {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kMaxMatsPerLaunch = 200;
+constexpr int kMaxMatsPerLaunch = 256;
 constexpr int kMaxC = 32768;
 
 struct UpdDesc {
@@ -55,17 +55,116 @@ struct UpdBatch {
     int32_t t_max;
     UpdDesc d[kMaxMatsPerLaunch];
 };
-static_assert(sizeof(UpdBatch) < 32000, "kernel parameter space");
+static_assert(sizeof(UpdBatch) <= 32764, "kernel parameter space");
+
+// q' = clamp(rint(W / s), -127, 127) with W / s the correctly rounded quotient. The quotient
+// matters only through its rounding to an integer, so it is first formed as W * rcp(s): that
+// product is within 1.6e-5 of W / s and the rounded quotient within 7.6e-6 (|W / s| <= 127.5),
+// so both round to the same integer unless the product lies within 2.3e-5 of a half-integer.
+// Only then (about 1 element in 8,000) is the exact division done.
+__device__ __forceinline__ float quant_code(float w, float sp, float rcp, bool fast)
+{
+    float qf;
+    const float y = __fmul_rn(w, rcp);
+    const float frac = y - floorf(y);
+    if (fast && fabsf(frac - 0.5f) >= 0x1p-14f) qf = rintf(y);
+    else qf = rintf(__fdiv_rn(w, sp));
+    return fminf(fmaxf(qf, -127.0f), 127.0f);
+}
+
+// Pass 1 of one 8-column chunk: rebuild, mix, Adam. Returns the new weights; stores moments.
+struct Chunk {
+    uint2 q;
+    float4 d0, d1, g0, g1, p0, p1;
+    uint4 m, v;
+};
+
+__device__ __forceinline__ void load_chunk(Chunk &k, const int8_t *qrow, const float *drow, const float *grow,
+                                           const float *prow, const uint16_t *mrow, const uint16_t *vrow,
+                                           int c0, bool partner, bool moments)
+{
+    k.q = __ldcs(reinterpret_cast<const uint2 *>(qrow + c0));
+    k.d0 = __ldcs(reinterpret_cast<const float4 *>(drow + c0));
+    k.d1 = __ldcs(reinterpret_cast<const float4 *>(drow + c0 + 4));
+    k.g0 = __ldcs(reinterpret_cast<const float4 *>(grow + c0));
+    k.g1 = __ldcs(reinterpret_cast<const float4 *>(grow + c0 + 4));
+    if (partner) {
+        k.p0 = __ldg(reinterpret_cast<const float4 *>(prow + c0));
+        k.p1 = __ldg(reinterpret_cast<const float4 *>(prow + c0 + 4));
+    } else {
+        k.p0 = k.p1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (moments) {
+        k.m = __ldcs(reinterpret_cast<const uint4 *>(mrow + c0));
+        k.v = __ldcs(reinterpret_cast<const uint4 *>(vrow + c0));
+    } else {
+        k.m = k.v = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
+
+struct AdamRow {
+    float sc, c_self, c_partner, beta1, beta2, omb1, omb2, bc1, bc2, eps, nlr, nlrwd, clip, wd;
+};
+
+// nan_sum stays exactly 0 while every new weight is finite (w - w is 0 for finite w, NaN for
+// inf or NaN, and a NaN survives every later addition); big tracks the largest moment, which
+// must stay below 65520 to be representable in fp16.
+__device__ __forceinline__ void adam_chunk(const Chunk &k, const AdamRow &a, float (&wn)[8], uint4 &mo,
+                                           uint4 &vo, float &amax, float &nan_sum, float &big)
+{
+    const float dl[8] = {k.d0.x, k.d0.y, k.d0.z, k.d0.w, k.d1.x, k.d1.y, k.d1.z, k.d1.w};
+    const float ga_[8] = {k.g0.x, k.g0.y, k.g0.z, k.g0.w, k.g1.x, k.g1.y, k.g1.z, k.g1.w};
+    const float gb_[8] = {k.p0.x, k.p0.y, k.p0.z, k.p0.w, k.p1.x, k.p1.y, k.p1.z, k.p1.w};
+    const uint32_t mw[4] = {k.m.x, k.m.y, k.m.z, k.m.w};
+    const uint32_t vw[4] = {k.v.x, k.v.y, k.v.z, k.v.w};
+    uint32_t mout[4], vout[4];
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+        const float2 mo2 = __half22float2(*reinterpret_cast<const __half2 *>(&mw[e2]));
+        const float2 vo2 = __half22float2(*reinterpret_cast<const __half2 *>(&vw[e2]));
+        float m1[2], v1[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int e = 2 * e2 + h;
+            const int8_t qe = static_cast<int8_t>(((e < 4 ? k.q.x : k.q.y) >> (8 * (e & 3))) & 0xFF);
+            const float W = __fmaf_rn(a.sc, (float)qe, dl[e]);
+            float ga = ga_[e], gb = gb_[e];
+            if (a.clip > 0.0f) {
+                ga = fminf(fmaxf(ga, -a.clip), a.clip);
+                gb = fminf(fmaxf(gb, -a.clip), a.clip);
+            }
+            const float gt = __fmaf_rn(a.c_partner, gb, __fmul_rn(a.c_self, ga));
+            const float mold = h ? mo2.y : mo2.x;
+            const float vold = h ? vo2.y : vo2.x;
+            m1[h] = __fmaf_rn(a.beta1, mold, __fmul_rn(a.omb1, gt));
+            v1[h] = __fmaf_rn(a.beta2, vold, __fmul_rn(a.omb2, __fmul_rn(gt, gt)));
+            const float u = __fdiv_rn(__fmul_rn(m1[h], a.bc1),
+                                      __fadd_rn(__fsqrt_rn(__fmul_rn(v1[h], a.bc2)), a.eps));
+            float Wn = __fmaf_rn(a.nlr, u, W);
+            if (a.wd != 0.0f) Wn = __fmaf_rn(a.nlrwd, W, Wn);
+            wn[e] = Wn;
+            amax = fmaxf(amax, fabsf(Wn));
+            nan_sum = __fadd_rn(nan_sum, __fsub_rn(Wn, Wn));
+            big = fmaxf(big, fmaxf(fabsf(m1[h]), v1[h]));
+        }
+        const __half2 mh = __floats2half2_rn(m1[0], m1[1]);
+        const __half2 vh = __floats2half2_rn(v1[0], v1[1]);
+        mout[e2] = *reinterpret_cast<const uint32_t *>(&mh);
+        vout[e2] = *reinterpret_cast<const uint32_t *>(&vh);
+    }
+    mo = make_uint4(mout[0], mout[1], mout[2], mout[3]);
+    vo = make_uint4(vout[0], vout[1], vout[2], vout[3]);
+}
 
 // One CTA owns one row at a time. Pass 1 streams the row's q, delta, gradient(s) and moments
-// through registers one 8-column chunk per thread per iteration, stores the new moments at once
-// and parks the new fp32 weight in shared memory (4*C bytes), so a thread needs few registers
-// and four CTAs share an SM; pass 2 requantises from shared memory.
-__global__ void __launch_bounds__(kThreads, 4)
+// through registers, UNROLL chunks of 8 columns per thread in flight, stores the new moments at
+// once and parks the new fp32 weight in shared memory (4*C bytes), so a thread needs few
+// registers and several CTAs share an SM; pass 2 requantises from shared memory.
+template <int UNROLL>
+__global__ void __launch_bounds__(kThreads, UNROLL == 1 ? 4 : 3)
 update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
 {
     extern __shared__ float4 wrow4[];                 // new weights of the current row
-    float *wrow = reinterpret_cast<float *>(wrow4);
     __shared__ int s_prefix[kMaxMatsPerLaunch + 1];
     __shared__ int scan_scratch[33];
     __shared__ uint32_t max_scratch[33];
@@ -83,9 +182,7 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         __syncthreads();
     }
     const int total = s_prefix[b.n];
-    const float nlr = -b.lr;
-    const float nlrwd = __fmul_rn(-b.lr, b.wd);
-    bool nonfinite = false;
+    float nan_sum = 0.0f, big = 0.0f;
 
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
         int lo = 0, hi = b.n - 1;
@@ -101,8 +198,21 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         const int t_old = d.slot_step[slot];
         const int t = t_old + 1;
         const int ti = t < b.t_max ? t : b.t_max;
-        const float bc1 = b.bc1[ti], bc2 = b.bc2[ti];
-        const float sc = d.s[r];
+        AdamRow a;
+        a.sc = d.s[r];
+        a.c_self = d.c_self;
+        a.c_partner = d.c_partner;
+        a.beta1 = b.beta1;
+        a.beta2 = b.beta2;
+        a.omb1 = b.omb1;
+        a.omb2 = b.omb2;
+        a.bc1 = b.bc1[ti];
+        a.bc2 = b.bc2[ti];
+        a.eps = b.eps;
+        a.nlr = -b.lr;
+        a.nlrwd = __fmul_rn(-b.lr, b.wd);
+        a.clip = b.clip;
+        a.wd = b.wd;
         const int C = d.C, nchunks = C >> 3;
         const int8_t *qrow = d.q + (size_t)r * C;
         const float *drow = d.delta + (size_t)r * C;
@@ -110,74 +220,37 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         const float *prow = d.pgrad + (size_t)(pslot < 0 ? 0 : pslot) * C;
         uint16_t *mrow = d.m + (size_t)slot * C;
         uint16_t *vrow = d.v + (size_t)slot * C;
+        const bool partner = pslot >= 0, moments = t_old > 0;
 
         // ---- pass 1: rebuild, mix, Adam; moments out, new weight to shared memory ----
         float amax = 0.0f;
-        for (int j = tid; j < nchunks; j += kThreads) {
-            const int c0 = j << 3;
-            const uint2 qv = __ldcs(reinterpret_cast<const uint2 *>(qrow + c0));
-            const float4 d0 = __ldcs(reinterpret_cast<const float4 *>(drow + c0));
-            const float4 d1 = __ldcs(reinterpret_cast<const float4 *>(drow + c0 + 4));
-            const float4 g0 = __ldcs(reinterpret_cast<const float4 *>(grow + c0));
-            const float4 g1 = __ldcs(reinterpret_cast<const float4 *>(grow + c0 + 4));
-            float4 p0 = make_float4(0.f, 0.f, 0.f, 0.f), p1 = p0;
-            if (pslot >= 0) {
-                p0 = __ldg(reinterpret_cast<const float4 *>(prow + c0));
-                p1 = __ldg(reinterpret_cast<const float4 *>(prow + c0 + 4));
-            }
-            uint4 mv = make_uint4(0u, 0u, 0u, 0u), vv = mv;
-            if (t_old > 0) {
-                mv = __ldcs(reinterpret_cast<const uint4 *>(mrow + c0));
-                vv = __ldcs(reinterpret_cast<const uint4 *>(vrow + c0));
-            }
-            const float dl[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-            const float ga_[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-            const float gb_[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-            const uint32_t mw[4] = {mv.x, mv.y, mv.z, mv.w};
-            const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-            uint32_t mout[4], vout[4];
-            float wn[8];
+        for (int j0 = tid; j0 < nchunks; j0 += kThreads * UNROLL) {
+            Chunk k[UNROLL];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const int8_t qe = static_cast<int8_t>(((e < 4 ? qv.x : qv.y) >> (8 * (e & 3))) & 0xFF);
-                const float W = __fmaf_rn(sc, (float)qe, dl[e]);
-                float ga = ga_[e], gb = gb_[e];
-                if (b.clip > 0.0f) {
-                    ga = fminf(fmaxf(ga, -b.clip), b.clip);
-                    gb = fminf(fmaxf(gb, -b.clip), b.clip);
-                }
-                const float gt = __fmaf_rn(d.c_partner, gb, __fmul_rn(d.c_self, ga));
-                const float m_old = __half2float(__ushort_as_half((uint16_t)(mw[e >> 1] >> (16 * (e & 1)))));
-                const float v_old = __half2float(__ushort_as_half((uint16_t)(vw[e >> 1] >> (16 * (e & 1)))));
-                const float m1 = __fmaf_rn(b.beta1, m_old, __fmul_rn(b.omb1, gt));
-                const float v1 = __fmaf_rn(b.beta2, v_old, __fmul_rn(b.omb2, __fmul_rn(gt, gt)));
-                const float u = __fdiv_rn(__fmul_rn(m1, bc1),
-                                          __fadd_rn(__fsqrt_rn(__fmul_rn(v1, bc2)), b.eps));
-                float Wn = __fmaf_rn(nlr, u, W);
-                if (b.wd != 0.0f) Wn = __fmaf_rn(nlrwd, W, Wn);
-                const uint16_t m16 = __half_as_ushort(__float2half_rn(m1));
-                const uint16_t v16 = __half_as_ushort(__float2half_rn(v1));
-                nonfinite |= !isfinite(Wn) || (v16 & 0x7C00u) == 0x7C00u || (m16 & 0x7C00u) == 0x7C00u;
-                if (e & 1) {
-                    mout[e >> 1] |= (uint32_t)m16 << 16;
-                    vout[e >> 1] |= (uint32_t)v16 << 16;
-                } else {
-                    mout[e >> 1] = m16;
-                    vout[e >> 1] = v16;
-                }
-                wn[e] = Wn;
-                amax = fmaxf(amax, fabsf(Wn));
+            for (int u = 0; u < UNROLL; ++u) {
+                const int j = j0 + u * kThreads;
+                if (j < nchunks) load_chunk(k[u], qrow, drow, grow, prow, mrow, vrow, j << 3, partner, moments);
             }
-            __stcs(reinterpret_cast<uint4 *>(mrow + c0), make_uint4(mout[0], mout[1], mout[2], mout[3]));
-            __stcs(reinterpret_cast<uint4 *>(vrow + c0), make_uint4(vout[0], vout[1], vout[2], vout[3]));
-            wrow4[2 * j] = make_float4(wn[0], wn[1], wn[2], wn[3]);
-            wrow4[2 * j + 1] = make_float4(wn[4], wn[5], wn[6], wn[7]);
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int j = j0 + u * kThreads;
+                if (j >= nchunks) break;
+                float wn[8];
+                uint4 mo, vo;
+                adam_chunk(k[u], a, wn, mo, vo, amax, nan_sum, big);
+                __stcs(reinterpret_cast<uint4 *>(mrow + (j << 3)), mo);
+                __stcs(reinterpret_cast<uint4 *>(vrow + (j << 3)), vo);
+                wrow4[2 * j] = make_float4(wn[0], wn[1], wn[2], wn[3]);
+                wrow4[2 * j + 1] = make_float4(wn[4], wn[5], wn[6], wn[7]);
+            }
         }
 
         // new per-row scale from the row absmax (non-negative floats order as unsigned ints);
         // the reduction's barriers also publish the shared-memory row to every thread
         const float rmax = __uint_as_float(block_max_u32(__float_as_uint(amax), max_scratch));
         const float sp = __fdiv_rn(rmax, 127.0f);
+        const float rcp = __frcp_rn(sp);
+        const bool fast = sp != 0.0f && isfinite(rcp);
 
         // ---- pass 2: requantise from shared memory, write q, delta and the live row ----
         int8_t *qout = d.q + (size_t)r * C;
@@ -189,26 +262,28 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
             const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
             uint32_t qo[2] = {0u, 0u};
             float dn[8];
-            uint32_t lo16[4];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float Wn = wv[e];
-                float qf = 0.0f, de = Wn;
+                float qf = 0.0f, de = wv[e];
                 if (sp != 0.0f) {
-                    qf = rintf(__fdiv_rn(Wn, sp));
-                    qf = fminf(fmaxf(qf, -127.0f), 127.0f);
-                    de = __fmaf_rn(-sp, qf, Wn);
+                    qf = quant_code(wv[e], sp, rcp, fast);
+                    de = __fmaf_rn(-sp, qf, wv[e]);
                 }
                 qo[e >> 2] |= ((uint32_t)(int)qf & 0xFFu) << (8 * (e & 3));
                 dn[e] = de;
-                const uint16_t lb = __bfloat16_as_ushort(__float2bfloat16_rn(Wn));
-                if (e & 1) lo16[e >> 1] |= (uint32_t)lb << 16; else lo16[e >> 1] = lb;
             }
             __stcs(reinterpret_cast<uint2 *>(qout + c0), make_uint2(qo[0], qo[1]));
             __stcs(reinterpret_cast<float4 *>(dout + c0), make_float4(dn[0], dn[1], dn[2], dn[3]));
             __stcs(reinterpret_cast<float4 *>(dout + c0 + 4), make_float4(dn[4], dn[5], dn[6], dn[7]));
-            if (lout)
-                __stcs(reinterpret_cast<uint4 *>(lout + c0), make_uint4(lo16[0], lo16[1], lo16[2], lo16[3]));
+            if (lout) {
+                const __nv_bfloat162 l0 = __floats2bfloat162_rn(wv[0], wv[1]);
+                const __nv_bfloat162 l1 = __floats2bfloat162_rn(wv[2], wv[3]);
+                const __nv_bfloat162 l2 = __floats2bfloat162_rn(wv[4], wv[5]);
+                const __nv_bfloat162 l3 = __floats2bfloat162_rn(wv[6], wv[7]);
+                __stcs(reinterpret_cast<uint4 *>(lout + c0),
+                       make_uint4(*reinterpret_cast<const uint32_t *>(&l0), *reinterpret_cast<const uint32_t *>(&l1),
+                                  *reinterpret_cast<const uint32_t *>(&l2), *reinterpret_cast<const uint32_t *>(&l3)));
+            }
         }
         if (tid == 0) {
             d.s[r] = sp;
@@ -216,7 +291,7 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         }
         __syncthreads();                 // the shared row is reused by the next item
     }
-    if (nonfinite) set_status(status, SF_STATUS_NONFINITE);
+    if (nan_sum != 0.0f || !(big < 65520.0f)) set_status(status, SF_STATUS_NONFINITE);
 }
 
 // 1/(1 - beta^t) for t = 0..t_max; beta^t as t successive fp64 products of the fp32 beta.
@@ -305,11 +380,16 @@ extern "C" int sf_sparse_update(const sf_matrix *mats, int n_mats, const sf_adam
     const int sms = sm_count();
     if (sms <= 0) return SF_ERR_NO_DEVICE;
     const size_t smem = (size_t)maxC * sizeof(float);
+#ifndef SF_UPDATE_UNROLL
+#define SF_UPDATE_UNROLL 1
+#endif
+    const int unroll = SF_UPDATE_UNROLL;
+    const void *fn = unroll == 2 ? (const void *)update_kernel<2> : (const void *)update_kernel<1>;
     if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return SF_ERR_CUDA;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, update_kernel, kThreads, smem) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem) != cudaSuccess ||
         per_sm <= 0)
         return SF_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
@@ -349,7 +429,10 @@ extern "C" int sf_sparse_update(const sf_matrix *mats, int n_mats, const sf_adam
             d.pgrad = a.partner >= 0 ? mats[a.partner].grad : nullptr;
             d.prow_slot = a.partner >= 0 ? mats[a.partner].mask.row_slot : nullptr;
         }
-        update_kernel<<<sms * per_sm, kThreads, smem, st>>>(b, dev_status);
+        if (unroll == 2)
+            update_kernel<2><<<sms * per_sm, kThreads, smem, st>>>(b, dev_status);
+        else
+            update_kernel<1><<<sms * per_sm, kThreads, smem, st>>>(b, dev_status);
         if (launch_status() != SF_OK) return SF_ERR_CUDA;
     }
     return SF_OK;

@@ -91,6 +91,39 @@ class SparseModel:
         return self.index[(p.layer, other)] + off
 
 
+def dw_launch_count(problems, group_bytes=320, prob_bytes=192, payload=32640, max_per_launch=96,
+                    max_per_group=8) -> int:
+    """Launches sf_masked_dw splits a call into: consecutive problems reading the same input form
+    a group, and groups are packed into kernel-parameter payloads of `payload` bytes, evenly.
+    problems: [(input identity, C)] in call order."""
+    groups = []
+    for key in problems:
+        if groups and groups[-1][0] == key and groups[-1][1] < max_per_group:
+            groups[-1][1] += 1
+        else:
+            groups.append([key, 1])
+    sizes = [group_bytes + n * prob_bytes for _, n in groups]
+    n_launch = max(1, -(-sum(sizes) // payload))
+    gi, li, launches = 0, 0, 0
+    while gi < len(groups):
+        left = sum(sizes[gi:])
+        target = -(-left // max(1, n_launch - li))
+        used, np_, g_end = 0, 0, gi
+        while g_end < len(groups):
+            add = sizes[g_end]
+            if g_end > gi and (used + add > payload or used >= target):
+                break
+            if g_end - gi + 1 > max_per_launch or np_ + groups[g_end][1] > max_per_launch:
+                break
+            used += add
+            np_ += groups[g_end][1]
+            g_end += 1
+        if g_end < len(groups) and li + 1 >= n_launch:
+            n_launch += 1
+        gi, li, launches = g_end, li + 1, launches + 1
+    return launches
+
+
 class StepPlan:
     """ABI argument arrays of one step over `model` for one set of input buffers.
 
@@ -123,6 +156,8 @@ class StepPlan:
                  for i, p in enumerate(model.projs)]
         self.n_dw = len(probs)
         self.dw_arr = (sf.sf_dw_problem * len(probs))(*probs)
+        self.dw_ws = torch.empty(max(L.sf_masked_dw_ws_bytes(self.dw_arr, self.n_dw), 1), dtype=torch.uint8,
+                                 device=model.device)
         structs = []
         if model.emb is not None:
             structs.append(sf.matrix_struct(model.emb))
@@ -130,6 +165,7 @@ class StepPlan:
             structs.append(sf.matrix_struct(p.mat, model.partner_index(i), 1.0, 0.0))
         self.upd_arr = (sf.sf_matrix * len(structs))(*structs)
         self.embed_ws = embed_ws
+        self.dw_launches = dw_launch_count([(id(inputs["A"][i]), p.mat.C) for i, p in enumerate(model.projs)])
         if model.emb is not None:
             self.emb_mask = model.emb.mask.struct()
 
@@ -152,7 +188,8 @@ class StepPlan:
                                           status, stream), "sf_mask_update")
 
     def dw(self, status, stream):
-        sf._check(self.lib.sf_masked_dw(self.dw_arr, self.n_dw, status, stream), "sf_masked_dw")
+        sf._check(self.lib.sf_masked_dw(self.dw_arr, self.n_dw, self.dw_ws.data_ptr(), self.dw_ws.numel(),
+                                        status, stream), "sf_masked_dw")
 
     def embed(self, status, stream):
         if self.model.emb is None:
@@ -173,9 +210,9 @@ class StepPlan:
         """Kernel launches one step issues (for the launch count of a timed region)."""
         def chunks(n, k):
             return (n + k - 1) // k
-        n_mask_batches = chunks(self.n_masks, 200)
+        n_mask_batches = chunks(self.n_masks, sf.SF_MASKS_PER_LAUNCH)
         n = 2 * n_mask_batches                       # accumulate + finalize per batch of masks
-        n += chunks(self.n_dw, sf.SF_DW_MAX_PER_LAUNCH)
+        n += 2 * self.dw_launches                   # gather + main kernel per launch
         n += 2 if self.model.emb is not None else 0
-        n += chunks(len(self.upd_arr), 200)
+        n += chunks(len(self.upd_arr), sf.SF_MATS_PER_LAUNCH)
         return n

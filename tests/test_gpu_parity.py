@@ -190,17 +190,24 @@ def _check_dw(case, ref=None):
             assert got[s].view(np.uint32).tolist() == [int(CANARY)] * case["C"], f"slot {s} written"
 
 
-def test_masked_dw_tiny_projection(sf):
+def _run_dw(sf, problems, mode, status=None):
+    ws = sf.dw_workspace(problems) if mode == "rows" else None
+    sf.sf_masked_dw(problems, status, ws=ws)
+
+
+@pytest.mark.parametrize("mode", ["tiles", "rows"])
+def test_masked_dw_tiny_projection(sf, mode):
     # W 256 x 512, T = 128: tile 0 full, tiles 3..7 empty, Bernoulli(0.03) rows elsewhere
     words = synth.tiny_projection_mask(0, 256)
     case = _dw_case(sf, 128, 256, 512, synth.rows_from_words(words), 0)
     status = sf.status_word()
-    sf.sf_masked_dw([sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])], status)
+    _run_dw(sf, [sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])], mode, status)
     _check_dw(case)
     assert host(status)[0] == 0
 
 
-def test_masked_dw_ragged_grouped_and_degenerate(sf):
+@pytest.mark.parametrize("mode", ["tiles", "rows"])
+def test_masked_dw_ragged_grouped_and_degenerate(sf, mode):
     # one launch: ragged T (not a multiple of 64), ragged C (last N-tile 8 wide), a ragged last
     # M-tile (7 active tiles), a full matrix, an all-empty mask and a zero-token problem
     g = synth.rng(3, "rows")
@@ -212,29 +219,80 @@ def test_masked_dw_ragged_grouped_and_degenerate(sf):
         _dw_case(sf, 333, 224, 1032, [0, 31, 32, 95, 96, 223], 5),
     ]
     status = sf.status_word()
-    sf.sf_masked_dw([sf.dw_problem(c["dXd"], c["Ad"], c["mask"], c["dW"]) for c in cases], status)
+    _run_dw(sf, [sf.dw_problem(c["dXd"], c["Ad"], c["mask"], c["dW"]) for c in cases], mode, status)
     for c in cases:
         _check_dw(c)
     assert host(status)[0] == 0
 
 
-def test_masked_dw_every_tile_position(sf):
+@pytest.mark.parametrize("mode", ["tiles", "rows"])
+def test_masked_dw_every_tile_position(sf, mode):
     # each of 40 tiles active with one row, in turn spread over M-tiles: catches slot/lane mixups
     R, C, T = 1280, 256, 96
     rows = np.array([32 * w + (w * 7) % 32 for w in range(R // 32)])
     case = _dw_case(sf, T, R, C, rows, 6)
-    sf.sf_masked_dw([sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])])
+    _run_dw(sf, [sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])], mode)
     _check_dw(case)
 
 
-def test_masked_dw_deterministic(sf):
+@pytest.mark.parametrize("mode", ["tiles", "rows"])
+def test_masked_dw_deterministic(sf, mode):
     words = synth.tiny_projection_mask(0, 256)
     case = _dw_case(sf, 1000, 256, 512, synth.rows_from_words(words), 8)
     p = [sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])]
-    sf.sf_masked_dw(p)
+    _run_dw(sf, p, mode)
     a = host(case["dW"]).copy()
-    sf.sf_masked_dw(p)
+    _run_dw(sf, p, mode)
     assert a.tobytes() == host(case["dW"]).tobytes()
+
+
+def test_masked_dw_groups_share_inputs_and_pick_their_mode(sf):
+    # q/k/v-like problems reading one A (a group: their scattered rows share 128-row tiles), a
+    # gate/up-like pair with whole active tiles (2 M-tiles either way, so tile mode is kept), and
+    # a problem whose active rows exceed its slots (row mode impossible -> tile mode).
+    T, C = 300, 520
+    A_bits = synth.normal_bf16(synth.rng(30, "act"), (T, C))
+    A = bf16_dev(A_bits)
+    cases, probs = [], []
+    g = synth.rng(30, "rows")
+    specs = [(512, np.sort(g.choice(512, 9, replace=False)), None, A_bits),
+             (512, np.sort(g.choice(512, 70, replace=False)), None, A_bits),
+             (1024, np.sort(g.choice(1024, 100, replace=False)), None, A_bits),
+             (256, np.arange(64, 128), None, None),
+             (256, np.arange(0, 128), None, "same"),
+             (384, np.sort(g.choice(384, 60, replace=False)), 20, None)]
+    shared2 = None
+    for i, (R, rows, cap, a_src) in enumerate(specs):
+        dX = synth.normal_bf16(synth.rng(30, "dx", i), (T, R))
+        if a_src is None:
+            a_bits = synth.normal_bf16(synth.rng(30, "act", i), (T, C))
+            a_dev = bf16_dev(a_bits)
+            shared2 = (a_bits, a_dev)
+        elif isinstance(a_src, str):
+            a_bits, a_dev = shared2
+        else:
+            a_bits, a_dev = A_bits, A
+        words = synth.words_from_rows(R, rows)
+        slot_cap = cap if cap is not None else min(R, len(rows) + 3)
+        mk = sf.Mask(R, slot_cap, DEV)
+        sf.sf_mask_init(mk)
+        sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_WORDS, u32_dev(words))], 0.01)
+        dW = _canary((slot_cap, C))
+        case = dict(dX=dX, A=a_bits, words=words, mask=mk, dW=dW, cap=slot_cap, C=C)
+        cases.append(case)
+        probs.append(sf.dw_problem(bf16_dev(dX), a_dev, mk, dW))
+    status = sf.status_word()
+    _run_dw(sf, probs, "rows", status)
+    for c in cases:
+        ref = orc.masked_dw(c["dX"], c["A"], c["words"])
+        mh = mask_host(c["mask"])
+        got = host(c["dW"])
+        for r in mh["rows"]:
+            s = mh["row_slot"][r]
+            if s < 0:
+                continue                       # no slot: no gradient is kept for this row
+            assert rel_err(got[s], ref[r], 1e-3) <= DW_TOL, r
+    assert host(status)[0] == 0
 
 
 # =============================================================================================
@@ -466,7 +524,8 @@ def test_tiny_projection_chain_three_steps(sf):
     for step in range(steps):
         dX = synth.normal_bf16(synth.rng(0, "dx", step), (T, R))
         A = synth.normal_bf16(synth.rng(0, "act", step), (T, C))
-        sf.sf_masked_dw([sf.dw_problem(bf16_dev(dX), bf16_dev(A), mat.mask, mat.grad)], status)
+        probs = [sf.dw_problem(bf16_dev(dX), bf16_dev(A), mat.mask, mat.grad)]
+        sf.sf_masked_dw(probs, status, ws=sf.dw_workspace(probs))
         sf.sf_sparse_update([sf.matrix_struct(mat)], hp, status)
         orc.update(st, orc.masked_dw(dX, A, words, np.zeros((R, C))).astype(np.float32), ohp)
     assert host(status)[0] == 0
@@ -479,3 +538,27 @@ def test_tiny_projection_chain_three_steps(sf):
     assert np.abs(Wg[rows] - Wo[rows]).max() <= tol
     inactive = np.setdiff1d(np.arange(R), rows)
     assert host(mat.q)[inactive].tobytes() == q0[inactive].tobytes()
+
+
+def test_update_flags_nonfinite_gradients_and_fp16_overflow(sf):
+    # Faults are planted on the host: a NaN in one active row's gradient, and in another run a
+    # gradient large enough that v = (1 - beta2) g^2 exceeds fp16's range. Both raise
+    # SF_STATUS_NONFINITE; a clean run does not.
+    R, C = 64, 256
+    W = synth.weights_f32(synth.rng(9, "weights"), R, C)
+    words = synth.words_from_rows(R, [3, 40])
+    hp = sf.AdamParams()
+    for case in ("clean", "nan", "overflow"):
+        st = orc.MatrixState(W)
+        mat = _state_from_oracle(sf, st, 8)
+        _set_words(sf, [(mat, words)])
+        grad = _grad_rows(9, 0, R, C)
+        if case == "nan":
+            grad[40, 17] = np.nan
+        elif case == "overflow":
+            grad[3, 5] = 1.0e4
+        _load_grad(mat, grad)
+        status = sf.status_word()
+        sf.sf_sparse_update([sf.matrix_struct(mat)], hp, status)
+        flagged = bool(int(host(status)[0]) & sf.SF_STATUS_NONFINITE)
+        assert flagged == (case != "clean"), case
