@@ -62,6 +62,8 @@ typedef void *sf_stream;               /* cudaStream_t */
  *   words[R/32]      uint32  the mask: bit i of words[w] is row 32w+i
  *   active_rows[R]   int32   active rows, ascending; the first counts[0] are valid
  *   active_tiles[R/32] int32 tiles holding an active row, ascending; first counts[1] valid
+ *   tile_rows[R/32]  int32   for the j-th active tile, the number of active rows in the tiles
+ *                            before it (the position of its first row in active_rows)
  *   row_slot[R]      int32   moment/gradient slot of each row, -1 for none
  *   free_slots[slot_cap] int32  stack of free slots (the top counts[2] entries)
  *   slot_step[slot_cap]  int32  Adam step count of each slot; 0 marks fresh (zero) moments
@@ -80,6 +82,7 @@ typedef struct sf_mask {
     uint32_t *words;
     int32_t  *active_rows;
     int32_t  *active_tiles;
+    int32_t  *tile_rows;
     int32_t  *row_slot;
     int32_t  *free_slots;
     int32_t  *slot_step;

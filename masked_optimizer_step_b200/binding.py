@@ -40,7 +40,7 @@ _F = ctypes.c_float
 
 class sf_mask(ctypes.Structure):
     _fields_ = [("R", _I32), ("slot_cap", _I32), ("charge", _P), ("accum", _P), ("words", _P),
-                ("active_rows", _P), ("active_tiles", _P), ("row_slot", _P), ("free_slots", _P),
+                ("active_rows", _P), ("active_tiles", _P), ("tile_rows", _P), ("row_slot", _P), ("free_slots", _P),
                 ("slot_step", _P), ("counts", _P)]
 
 
@@ -146,6 +146,7 @@ class Mask:
         self.words = torch.zeros(R // 32, **i32)
         self.active_rows = torch.zeros(R, **i32)
         self.active_tiles = torch.zeros(R // 32, **i32)
+        self.tile_rows = torch.zeros(R // 32, **i32)
         self.row_slot = torch.full((R,), -1, **i32)
         self.free_slots = torch.zeros(max(slot_cap, 1), **i32)
         self.slot_step = torch.zeros(max(slot_cap, 1), **i32)
@@ -153,7 +154,7 @@ class Mask:
 
     def struct(self) -> sf_mask:
         return sf_mask(self.R, self.slot_cap, _ptr(self.charge), _ptr(self.accum), _ptr(self.words),
-                       _ptr(self.active_rows), _ptr(self.active_tiles), _ptr(self.row_slot),
+                       _ptr(self.active_rows), _ptr(self.active_tiles), _ptr(self.tile_rows), _ptr(self.row_slot),
                        _ptr(self.free_slots), _ptr(self.slot_step), _ptr(self.counts))
 
 

@@ -54,37 +54,58 @@ constexpr int TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int kThreads = 192;
 constexpr size_t kSmemBytes = (size_t)STAGES * STAGE_BYTES + 1024;   // + alignment slack
 constexpr int kMaxPerGroup = 8;
-constexpr int kInfoInts = 16;           // per group: mode, total rows, row prefix [kMaxPerGroup+1]
 constexpr int kGatherTokens = 32;       // tokens per gather CTA
 constexpr int kGatherThreads = 256;
 
 struct alignas(64) DwProb {
-    CUtensorMap tm_dx;           // dX: dims {R, T}, box {32, 64}, 64-byte swizzle
-    const uint16_t *dx;
+    CUtensorMap tm_dx;           // dX: dims {R, T}, box {32, 64}, 64-byte swizzle (tile mode)
     const int32_t *active_tiles;
-    const int32_t *active_rows;
     const int32_t *counts;
     const int32_t *row_slot;
     float *dW;
-    int32_t ld_dx, ld_dw, R, group;
+    int64_t ld_dw;
 };
 
 struct alignas(64) DwGroup {
     CUtensorMap tm_a;            // A: dims {C, T}, box {64, 64}, 128-byte swizzle
     CUtensorMap tm_g;            // gathered rows: dims {mcap, T}, box {32, 64}, 64-byte swizzle
-    uint16_t *dxg;               // gathered rows, T x mcap bf16 (null: tile mode only)
-    int32_t *info;               // device: [0] mode (1 = rows), [1] rows, [2..] row prefix
+    const int32_t *info;         // device: [0] mode (1 = rows), [1] gathered rows (null: tiles only)
+    const int32_t *rowmap;       // device: per gathered row, (slot << 3) | problem, or -1
     int32_t first, count, C, T, n_ntiles, mcap;
 };
-
-constexpr int kParamBudget = 32764;
 
 struct DwBatch {
     int32_t n_prob, n_group;
     // variable-length payload: n_group DwGroup then n_prob DwProb
     alignas(64) unsigned char payload[32640];
 };
-static_assert(sizeof(DwBatch) <= kParamBudget, "kernel parameter space");
+static_assert(sizeof(DwBatch) <= 32764, "kernel parameter space");
+
+// The gather pass has its own, lean parameters (no tensor maps), so one launch covers a call.
+struct GatherProb {
+    const uint16_t *dx;
+    const int32_t *active_rows;
+    const int32_t *counts;
+    const int32_t *row_slot;
+    int64_t ld_dx;
+};
+
+struct GatherGroup {
+    uint16_t *dxg;
+    int32_t *info;
+    int32_t *rowmap;
+    int32_t first, count, T, mcap;
+};
+
+constexpr int kMaxGatherGroups = 192;
+constexpr int kMaxGatherProbs = 384;
+
+struct GatherBatch {
+    int32_t n_group, n_prob;
+    GatherGroup g[kMaxGatherGroups];
+    GatherProb p[kMaxGatherProbs];
+};
+static_assert(sizeof(GatherBatch) <= 32764, "kernel parameter space");
 
 __device__ __forceinline__ const DwGroup &grp(const DwBatch &b, int g)
 {
@@ -112,74 +133,68 @@ constexpr uint32_t kLayoutSW64 = 4;
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                             ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
-// Mode and size of a group, from the live masks. Every reader computes the same answer.
-struct GroupPlan {
-    int rows_mode;      // 1: row mode
-    int m_tiles;        // M-tiles of the group in its mode
-    int total_rows;     // active rows of all problems of the group
-};
-
-__device__ __forceinline__ GroupPlan plan_group(const DwBatch &b, const DwGroup &g)
+// Row mode when the group's active rows fit the scratch and need fewer 128-row tiles than the
+// mask tiles do. Every reader computes the same answer from the same counts.
+__device__ __forceinline__ bool choose_rows(int rows, int tiles_mt, int mcap)
 {
-    int rows = 0, tiles_mt = 0;
-    for (int k = 0; k < g.count; ++k) {
-        const DwProb &p = prb(b, g.first + k);
-        rows += p.counts[0];
-        tiles_mt += (p.counts[1] + 3) >> 2;
-    }
-    const int rows_mt = (rows + BM - 1) / BM;
-    GroupPlan pl;
-    pl.rows_mode = g.dxg != nullptr && rows <= g.mcap && rows_mt < tiles_mt;
-    pl.m_tiles = pl.rows_mode ? rows_mt : tiles_mt;
-    pl.total_rows = rows;
-    return pl;
+    return mcap > 0 && rows <= mcap && (rows + BM - 1) / BM < tiles_mt;
 }
 
 // ------------------------------------ gather kernel ------------------------------------
-// Row mode only: dxg[t, k] = dX_p[t, active_rows_p[k - prefix_p]] for the group's k-th active
-// row. One CTA per (group, 32 tokens); the first CTA of a group also records the plan, which the
-// main kernel (next on the stream) reads.
+// Row mode: dxg[t, k] = dX_p[t, r] for the group's k-th active row r (problems in call order,
+// rows ascending), and rowmap[k] = (slot(r) << 3) | p. One CTA per (group, 32 tokens); a thread
+// takes a gathered row and issues its 32 token loads back to back. The reads are single
+// elements spread over dX, so what bounds this pass is how many requests are in flight; many
+// small independent loads per thread measured faster than fewer 64-byte tile-segment loads.
+// Consecutive threads take consecutive gathered rows, so the writes coalesce. The first CTA of
+// a group records the mode and the row map, which the main kernel (next on the stream) reads.
 __global__ void __launch_bounds__(kGatherThreads)
-dw_gather_kernel(const __grid_constant__ DwBatch b, int blocks_per_group)
+dw_gather_kernel(const __grid_constant__ GatherBatch b, int blocks_per_group)
 {
     const int gi = blockIdx.x / blocks_per_group;
     const int tb = blockIdx.x - gi * blocks_per_group;
-    const DwGroup &g = grp(b, gi);
-    if (g.dxg == nullptr) return;
-    const GroupPlan pl = plan_group(b, g);
-    __shared__ int prefix[kMaxPerGroup + 1];
+    const GatherGroup &g = b.g[gi];
+    __shared__ int row_pre[kMaxPerGroup + 1];
+    __shared__ int s_rows_mode;
     if (threadIdx.x == 0) {
-        int acc = 0;
+        int rows = 0, tiles_mt = 0;
         for (int k = 0; k < g.count; ++k) {
-            prefix[k] = acc;
-            acc += prb(b, g.first + k).counts[0];
+            const GatherProb &p = b.p[g.first + k];
+            row_pre[k] = rows;
+            rows += p.counts[0];
+            tiles_mt += (p.counts[1] + 3) >> 2;
         }
-        prefix[g.count] = acc;
+        row_pre[g.count] = rows;
+        s_rows_mode = choose_rows(rows, tiles_mt, g.mcap);
         if (tb == 0) {
-            g.info[0] = pl.rows_mode;
-            g.info[1] = acc;
-            for (int k = 0; k <= g.count; ++k) g.info[2 + k] = prefix[k];
+            g.info[0] = s_rows_mode;
+            g.info[1] = rows;
         }
     }
     __syncthreads();
-    if (!pl.rows_mode) return;
+    if (!s_rows_mode) return;
     const int t0 = tb * kGatherTokens;
     const int nt = min(g.T - t0, kGatherTokens);
-    if (nt <= 0) return;
-    for (int k = threadIdx.x; k < pl.total_rows; k += kGatherThreads) {
-        int p = 0;
-        while (p + 1 < g.count && prefix[p + 1] <= k) ++p;
-        const DwProb &pr = prb(b, g.first + p);
-        const int r = pr.active_rows[k - prefix[p]];
-        const uint16_t *src = pr.dx + (size_t)t0 * pr.ld_dx + r;
+    const int rows = row_pre[g.count];
+    for (int k = threadIdx.x; k < rows; k += kGatherThreads) {
+        int q = 0;
+        while (q + 1 < g.count && row_pre[q + 1] <= k) ++q;
+        const GatherProb &p = b.p[g.first + q];
+        const int r = p.active_rows[k - row_pre[q]];
+        if (tb == 0) {
+            const int slot = p.row_slot[r];
+            g.rowmap[k] = slot >= 0 ? (slot << 3) | q : -1;
+        }
+        if (nt <= 0) continue;
+        const uint16_t *src = p.dx + (size_t)t0 * p.ld_dx + r;
         uint16_t *dst = g.dxg + (size_t)t0 * g.mcap + k;
         uint16_t v[kGatherTokens];
 #pragma unroll
-        for (int j = 0; j < kGatherTokens; ++j)
-            if (j < nt) v[j] = __ldcs(src + (size_t)j * pr.ld_dx);
+        for (int t = 0; t < kGatherTokens; ++t)
+            if (t < nt) v[t] = __ldcs(src + (size_t)t * p.ld_dx);
 #pragma unroll
-        for (int j = 0; j < kGatherTokens; ++j)
-            if (j < nt) dst[(size_t)j * g.mcap] = v[j];
+        for (int t = 0; t < kGatherTokens; ++t)
+            if (t < nt) dst[(size_t)t * g.mcap] = v[t];
     }
 }
 
@@ -244,14 +259,14 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
         int units = 0;
         if (tid < b.n_group) {
             const DwGroup &g = grp(b, tid);
-            const GroupPlan pl = plan_group(b, g);
-            sp.rows_mode[tid] = pl.rows_mode;
-            units = pl.m_tiles * g.n_ntiles;
             int acc = 0;
             for (int k = 0; k < g.count; ++k) {
                 sp.mt_prefix[g.first + k] = acc;
                 acc += (prb(b, g.first + k).counts[1] + 3) >> 2;
             }
+            const int rows_mode = g.info != nullptr && g.info[0] != 0;
+            sp.rows_mode[tid] = rows_mode;
+            units = (rows_mode ? (g.info[1] + BM - 1) / BM : acc) * g.n_ntiles;
         }
         int total;
         const int off = block_exclusive_scan(units, scan_scratch, &total);
@@ -399,10 +414,11 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             if (x.rows_mode) {
                 const int k = x.mt * BM + quad * 32 + lane;
                 if (k < g.info[1]) {
-                    int q = 0;
-                    while (q + 1 < g.count && g.info[2 + q + 1] <= k) ++q;
-                    p = &prb(b, g.first + q);
-                    slot = p->row_slot[p->active_rows[k - g.info[2 + q]]];
+                    const int e = g.rowmap[k];
+                    if (e >= 0) {
+                        p = &prb(b, g.first + (e & 7));
+                        slot = e >> 3;
+                    }
                 }
             } else {
                 p = &prb(b, x.p);
@@ -494,12 +510,14 @@ bool encode_bf16(CUtensorMap *m, const void *base, int width, int T, int64_t ld,
 struct HostGroup {
     int first, count;
     int mcap;                    // gathered-row capacity (multiple of 32)
-    size_t ws_off;               // byte offset of the group's scratch (info block, then rows)
+    size_t ws_off;               // byte offset of the group's scratch: info, row map, rows
 };
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-constexpr size_t kInfoBytes = 256;      // info block, padded so the rows start 256-aligned
+constexpr size_t kInfoBytes = 256;
+
+size_t rowmap_bytes(int mcap) { return round_up((size_t)mcap * sizeof(int32_t), 256); }
 
 int plan_groups(const sf_dw_problem *probs, int n, HostGroup *out, size_t *ws_total)
 {
@@ -517,7 +535,8 @@ int plan_groups(const sf_dw_problem *probs, int n, HostGroup *out, size_t *ws_to
         for (int k = i; k < j; ++k) cap += (size_t)probs[k].mask.slot_cap;
         g.mcap = (int)round_up(cap, 32);
         g.ws_off = off;
-        off += kInfoBytes + round_up((size_t)(probs[i].T > 0 ? probs[i].T : 0) * g.mcap * 2, 256);
+        off += kInfoBytes + rowmap_bytes(g.mcap) +
+               round_up((size_t)(probs[i].T > 0 ? probs[i].T : 0) * g.mcap * 2, 256);
         i = j;
     }
     *ws_total = off;
@@ -550,12 +569,13 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
         int rc = check_mask(p.mask);
         if (rc != SF_OK) return rc;
         if (p.T < 0 || p.C <= 0 || (p.C & 7) || !p.dW) return SF_ERR_ARG;
-        if (p.ld_dw < p.C || p.ld_dw > INT32_MAX) return SF_ERR_ARG;
+        if (p.ld_dw < p.C) return SF_ERR_ARG;
         if ((p.ld_dw & 3) || !aligned16(p.dW)) return SF_ERR_ALIGN;
         if (p.T > 0) {                       // dX and A are read only when there are tokens
-            if (!p.dX || !p.A || p.ld_dx < p.mask.R || p.ld_a < p.C || p.ld_dx > INT32_MAX) return SF_ERR_ARG;
+            if (!p.dX || !p.A || p.ld_dx < p.mask.R || p.ld_a < p.C) return SF_ERR_ARG;
             if ((p.ld_dx & 7) || (p.ld_a & 7) || !aligned16(p.dX) || !aligned16(p.A)) return SF_ERR_ALIGN;
         }
+        if ((long long)p.mask.slot_cap * 8 > INT32_MAX) return SF_ERR_UNSUPPORTED;   // row map packing
     }
     if (n == 0) return SF_OK;
     HostGroup *groups = new HostGroup[n];
@@ -571,7 +591,45 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
                                             (int)kSmemBytes) != cudaSuccess)
         rc = SF_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
-    // Split the groups over as few launches as the parameter space allows, evenly by size.
+    auto scratch = [&](const HostGroup &hg) { return static_cast<uint8_t *>(ws) + hg.ws_off; };
+    auto row_ok = [&](const HostGroup &hg) { return use_ws && probs[hg.first].T > 0 && hg.mcap > 0; };
+
+    // ---- gather pass: every group of the call, in as few launches as the parameters allow ----
+    GatherBatch *gb = (rc == SF_OK && use_ws) ? new GatherBatch : nullptr;
+    for (int gi = 0; gb && rc == SF_OK && gi < ng;) {
+        memset(gb, 0, sizeof(*gb));
+        int tok_blocks = 1;
+        while (gi < ng && gb->n_group < kMaxGatherGroups && gb->n_prob + groups[gi].count <= kMaxGatherProbs) {
+            const HostGroup &hg = groups[gi++];
+            if (!row_ok(hg)) continue;
+            GatherGroup &g = gb->g[gb->n_group++];
+            uint8_t *base = scratch(hg);
+            g.info = reinterpret_cast<int32_t *>(base);
+            g.rowmap = reinterpret_cast<int32_t *>(base + kInfoBytes);
+            g.dxg = reinterpret_cast<uint16_t *>(base + kInfoBytes + rowmap_bytes(hg.mcap));
+            g.first = gb->n_prob;
+            g.count = hg.count;
+            g.T = probs[hg.first].T;
+            g.mcap = hg.mcap;
+            tok_blocks = max(tok_blocks, (g.T + kGatherTokens - 1) / kGatherTokens);
+            for (int q = 0; q < hg.count; ++q) {
+                const sf_dw_problem &p = probs[hg.first + q];
+                GatherProb &d = gb->p[gb->n_prob++];
+                d.dx = static_cast<const uint16_t *>(p.dX);
+                d.active_rows = p.mask.active_rows;
+                d.counts = p.mask.counts;
+                d.row_slot = p.mask.row_slot;
+                d.ld_dx = p.ld_dx;
+            }
+        }
+        if (gb->n_group > 0) {
+            dw_gather_kernel<<<gb->n_group * tok_blocks, kGatherThreads, 0, st>>>(*gb, tok_blocks);
+            if (launch_status() != SF_OK) rc = SF_ERR_CUDA;
+        }
+    }
+    delete gb;
+
+    // ---- main pass: groups split over launches so that each launch's parameters fit ----
     const size_t payload = sizeof(DwBatch::payload);
     size_t all = 0;
     for (int k = 0; k < ng; ++k) all += launch_bytes(groups[k]);
@@ -602,7 +660,6 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
         DwProb *pd = reinterpret_cast<DwProb *>(batch->payload + (size_t)batch->n_group * sizeof(DwGroup));
         long long max_units = 0;
         int pi = 0;
-        int tok_blocks = 1;
         for (int k = gi; k < g_end && rc == SF_OK; ++k) {
             const HostGroup &hg = groups[k];
             const sf_dw_problem &p0 = probs[hg.first];
@@ -616,13 +673,13 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
             g.T = p0.T;
             g.n_ntiles = (p0.C + BN - 1) / BN;
             g.mcap = hg.mcap;
-            if (use_ws && p0.T > 0 && hg.mcap > 0) {
-                uint8_t *base = static_cast<uint8_t *>(ws) + hg.ws_off;
-                g.info = reinterpret_cast<int32_t *>(base);
-                g.dxg = reinterpret_cast<uint16_t *>(base + kInfoBytes);
-                if (!encode_bf16(&g.tm_g, g.dxg, hg.mcap, p0.T, hg.mcap, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+            if (row_ok(hg)) {
+                uint8_t *base = scratch(hg);
+                g.info = reinterpret_cast<const int32_t *>(base);
+                g.rowmap = reinterpret_cast<const int32_t *>(base + kInfoBytes);
+                const void *dxg = base + kInfoBytes + rowmap_bytes(hg.mcap);
+                if (!encode_bf16(&g.tm_g, dxg, hg.mcap, p0.T, hg.mcap, 32, CU_TENSOR_MAP_SWIZZLE_64B))
                     rc = SF_ERR_CUDA;
-                tok_blocks = max(tok_blocks, (p0.T + kGatherTokens - 1) / kGatherTokens);
             }
             long long tiles_mt = 0;
             for (int q = 0; q < hg.count; ++q, ++pi) {
@@ -632,25 +689,16 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
                 if (!encode_bf16(&d.tm_dx, dx, p.mask.R, p.T, p.T > 0 ? p.ld_dx : p.mask.R, 32,
                                  CU_TENSOR_MAP_SWIZZLE_64B))
                     rc = SF_ERR_CUDA;
-                d.dx = static_cast<const uint16_t *>(p.dX);
                 d.active_tiles = p.mask.active_tiles;
-                d.active_rows = p.mask.active_rows;
                 d.counts = p.mask.counts;
                 d.row_slot = p.mask.row_slot;
                 d.dW = p.dW;
-                d.ld_dx = (int32_t)p.ld_dx;
-                d.ld_dw = (int32_t)p.ld_dw;
-                d.R = p.mask.R;
-                d.group = k - gi;
+                d.ld_dw = p.ld_dw;
                 tiles_mt += (p.mask.R / 32 + 3) / 4;
             }
             max_units += tiles_mt * g.n_ntiles;
         }
         if (rc != SF_OK) break;
-        if (use_ws) {
-            dw_gather_kernel<<<batch->n_group * tok_blocks, kGatherThreads, 0, st>>>(*batch, tok_blocks);
-            if (launch_status() != SF_OK) { rc = SF_ERR_CUDA; break; }
-        }
         const int grid = (int)(max_units < sms ? max_units : sms);
         if (grid > 0) {
             masked_dw_kernel<<<grid, kThreads, kSmemBytes, st>>>(*batch, dev_status);

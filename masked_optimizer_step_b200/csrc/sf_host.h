@@ -24,7 +24,7 @@ inline int launch_status()
 inline int check_mask(const sf_mask &m)
 {
     if (m.R <= 0 || (m.R & 31) || m.slot_cap < 0 || m.slot_cap > m.R) return SF_ERR_ARG;
-    if (!m.charge || !m.accum || !m.words || !m.active_rows || !m.active_tiles || !m.row_slot ||
+    if (!m.charge || !m.accum || !m.words || !m.active_rows || !m.active_tiles || !m.tile_rows || !m.row_slot ||
         !m.counts || !m.slot_step || (!m.free_slots && m.slot_cap > 0))
         return SF_ERR_ARG;
     return SF_OK;

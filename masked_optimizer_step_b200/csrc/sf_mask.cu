@@ -38,6 +38,7 @@ struct MaskDesc {
     uint32_t *words;
     int32_t *active_rows;
     int32_t *active_tiles;
+    int32_t *tile_rows;
     int32_t *row_slot;
     int32_t *free_slots;
     int32_t *slot_step;
@@ -270,7 +271,10 @@ mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *s
         int j = 0;
         for (uint32_t bits = word; bits; bits &= bits - 1)
             d.active_rows[rb + j++] = (w << 5) + __ffs(bits) - 1;
-        if (word) d.active_tiles[s_tiles + toff] = w;
+        if (word) {
+            d.active_tiles[s_tiles + toff] = w;
+            d.tile_rows[s_tiles + toff] = rb;
+        }
         if (w < nw) d.words[w] = word;
         __syncthreads();
         if (tid == 0) {
@@ -302,6 +306,7 @@ __global__ void mask_init_kernel(sf_mask m)
         if ((i & 31) == 0) {
             m.words[i >> 5] = 0u;
             m.active_tiles[i >> 5] = 0;
+            m.tile_rows[i >> 5] = 0;
         }
     }
     if (i < m.slot_cap) {
@@ -389,6 +394,7 @@ extern "C" int sf_mask_update(const sf_mask *masks, const sf_mask_src *srcs, int
             d.words = m.words;
             d.active_rows = m.active_rows;
             d.active_tiles = m.active_tiles;
+            d.tile_rows = m.tile_rows;
             d.row_slot = m.row_slot;
             d.free_slots = m.free_slots;
             d.slot_step = m.slot_step;

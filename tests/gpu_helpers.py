@@ -35,6 +35,7 @@ def mask_host(mask):
         words=host(mask.words).view(np.uint32),
         rows=host(mask.active_rows)[: c[0]],
         tiles=host(mask.active_tiles)[: c[1]],
+        tile_rows=host(mask.tile_rows)[: c[1]],
         counts=c,
         row_slot=host(mask.row_slot),
         slot_step=host(mask.slot_step),
@@ -43,8 +44,12 @@ def mask_host(mask):
 
 
 def check_slot_invariants(mh, slot_cap):
-    """Every active row holds a distinct slot (or none after overflow); nothing else holds one."""
+    """Every active row holds a distinct slot (or none after overflow); nothing else holds one.
+    Also: tile_rows[j] is the position in active_rows of the first row of the j-th active tile."""
     R = mh["row_slot"].size
+    for j, w in enumerate(mh["tiles"]):
+        assert mh["rows"][mh["tile_rows"][j]] // 32 == w
+        assert mh["tile_rows"][j] == 0 or mh["rows"][mh["tile_rows"][j] - 1] // 32 < w
     active = np.zeros(R, bool)
     active[mh["rows"]] = True
     slots = mh["row_slot"]
