@@ -30,6 +30,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse step ms & active-row updates/s at 7B shape, 1% active; % of roofline"
+
+# DRAM traffic per layer of each stage (dram__bytes_read.sum + dram__bytes_write.sum), measured
+# with ncu on the 2-layer case of the default workload (scattered masks, 2,048 tokens) and
+# scaled by the layer count; it applies to that workload only.
+TRAFFIC_PER_LAYER = {"masks": (348.56e6 + 3.85e6 + 1.08e6) / 2,
+                     "masked_dw": (203.92e6 + 8.32e6 + 173.74e6 + 3.98e6) / 2}
 UNIT = "active-row updates/s"
 SEED = 3
 
@@ -54,6 +60,20 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def reduce_over_ranks(ms: float, units: float, device="cpu"):
+    """Whole-job timing over ranks: the slowest rank's time (max) and every rank's work (sum).
+    Identity when no process group is running."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(ms), float(units)
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([float(units)], device=device, dtype=torch.float64)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(u[0])
 
 
 def workload_config(args):
@@ -395,15 +415,7 @@ def main():
     rows_updated = sum(w["rows_updated"] for w in work)
     dev_status = int(status.cpu()[0])
 
-    max_ms = ms_total
-    total_rows = rows_updated
-    if world > 1:
-        t = torch.tensor([ms_total], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        max_ms = float(t[0])
-        r = torch.tensor([rows_updated], device=device, dtype=torch.float64)
-        dist.all_reduce(r, op=dist.ReduceOp.SUM)
-        total_rows = float(r[0])
+    max_ms, total_rows = reduce_over_ranks(ms_total, rows_updated, device)
     value = total_rows / (max_ms / 1000.0)
 
     # ---- rooflines of each stage ----
@@ -454,8 +466,15 @@ def main():
                       "algorithmic_gb_per_step": step_bytes / args.steps / 1e9}
     dominant = max(("masks", "masked_dw", "sparse_update"), key=lambda s: stages[s]["ms_per_step"])
     d = stages[dominant]
+    traffic = None
+    if args.masks == "scattered" and args.tokens == 2048 and dominant in TRAFFIC_PER_LAYER:
+        traffic = TRAFFIC_PER_LAYER[dominant] * args.layers
+    kernels = {"masks": "sf_mask_update: mask_accum_kernel + mask_finalize_kernel",
+               "masked_dw": "sf_masked_dw: dw_gather_kernel + 3 x masked_dw_kernel",
+               "sparse_update": "sf_sparse_update: update_kernel"}
     roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-                "frac": d["frac"], "traffic": None, "kernel": dominant, "peak_source": peak_src,
+                "frac": d["frac"], "traffic": traffic, "traffic_unit": "bytes per step (one call)",
+                "kernel": kernels[dominant], "peak_source": peak_src,
                 "peak_kind": "sustained bf16 (kernel timed inside a long step)" if d["bound"] == "tensor" else "hbm copy",
                 "algorithmic": d["algorithmic"]}
 
@@ -562,13 +581,7 @@ def run_e2e(args, model, banks, plans, hp, tok_dev, prior, stream, device, world
     torch.cuda.synchronize()
     secs = time.perf_counter() - t0
     rows = K * sum(int(c[0]) - int(c[3]) for c in model.counts.cpu().numpy())
-    if world > 1:
-        t = torch.tensor([secs], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        secs = float(t[0])
-        r = torch.tensor([rows], device=device, dtype=torch.float64)
-        dist.all_reduce(r, op=dist.ReduceOp.SUM)
-        rows = float(r[0])
+    secs, rows = reduce_over_ranks(secs, rows, device)
     for p in plans:                        # restore the resident token buffers
         p.set_tokens(tok_dev[prior])
     return {"value": rows / secs, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
