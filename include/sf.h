@@ -49,7 +49,7 @@ extern "C" {
 /* ---- device status bits (OR-ed into *dev_status) --------------------------------------- */
 #define SF_STATUS_SLOT_OVERFLOW  0x1u  /* an active row found no free moment slot; it is not updated */
 #define SF_STATUS_NONFINITE      0x2u  /* a non-finite gradient, moment or weight was produced */
-#define SF_STATUS_BAD_TOKEN      0x4u  /* a token id outside [0, R) was ignored */
+#define SF_STATUS_BAD_TOKEN      0x4u  /* a token or row id outside [0, R) was ignored */
 #define SF_STATUS_WAIT_TIMEOUT   0x8u  /* a kernel gave up a bounded wait and skipped its work */
 
 typedef void *sf_stream;               /* cudaStream_t */
@@ -257,6 +257,37 @@ int sf_adam_tables(float beta1, float beta2, int t_max, float *bc1, float *bc2,
 
 int sf_sparse_update(const sf_matrix *mats /* host [n_mats] */, int n_mats,
                      const sf_adam *hp /* host */, uint32_t *dev_status, sf_stream stream);
+
+/* ---- sf_checkpoint_save / sf_checkpoint_restore: section 2.6, "Checkpoint and rewind" -----
+ * The optimizer keeps a checkpoint of the active rows only, so a checkpoint costs no more than
+ * the active set, and restores it when the loss rebounds (the policy that decides when is host
+ * logic). A checkpoint of one matrix is a snapshot, at save time, of each active row (ascending):
+ *   rows[k] the row, q[k*C..] int8, s[k], delta[k*C..] fp32, m, v[k*C..] fp16 bits (zeros for a
+ *   row without a slot), step[k] its Adam step count; *count the rows saved (device).
+ * Buffers hold `cap` rows; a save with more active rows keeps the first cap and sets
+ * SF_STATUS_SLOT_OVERFLOW. Restore writes q, s and delta of every saved row back and rebuilds its
+ * live row (bf16 of fma(s, q, delta)); moments and step count go back only to rows that hold a
+ * slot now (moments exist only for active rows). Rows not in the checkpoint are untouched.
+ * Restore reads at most cap rows (a larger *count is clamped); a saved row id outside [0, R) is
+ * skipped and sets SF_STATUS_BAD_TOKEN. `mats` and `ck` are host arrays of n entries (same order). Requirements: C a multiple of 16,
+ * all row buffers 16-byte aligned. Errors: SF_ERR_ARG, SF_ERR_ALIGN.
+ */
+typedef struct sf_checkpoint {
+    int32_t   cap;
+    int32_t  *count;
+    int32_t  *rows;
+    int8_t   *q;
+    float    *s;
+    float    *delta;
+    uint16_t *m;
+    uint16_t *v;
+    int32_t  *step;
+} sf_checkpoint;
+
+int sf_checkpoint_save(const sf_matrix *mats /* host [n] */, const sf_checkpoint *ck /* host [n] */,
+                       int n, uint32_t *dev_status, sf_stream stream);
+int sf_checkpoint_restore(const sf_matrix *mats /* host [n] */, const sf_checkpoint *ck /* host [n] */,
+                          int n, uint32_t *dev_status, sf_stream stream);
 
 /* ---- helpers (not on the hot path) ------------------------------------------------------ */
 

@@ -59,6 +59,11 @@ class sf_matrix(ctypes.Structure):
                 ("grad", _P), ("live", _P)]
 
 
+class sf_checkpoint(ctypes.Structure):
+    _fields_ = [("cap", _I32), ("count", _P), ("rows", _P), ("q", _P), ("s", _P), ("delta", _P),
+                ("m", _P), ("v", _P), ("step", _P)]
+
+
 class sf_adam(ctypes.Structure):
     _fields_ = [("lr", _F), ("beta1", _F), ("beta2", _F), ("eps", _F), ("one_minus_b1", _F),
                 ("one_minus_b2", _F), ("wd", _F), ("clip", _F), ("bc1", _P), ("bc2", _P),
@@ -97,6 +102,9 @@ def load():
     L.sf_sparse_update.argtypes = [ctypes.POINTER(sf_matrix), ctypes.c_int, ctypes.POINTER(sf_adam),
                                    _P, _P]
     L.sf_quantize_init.argtypes = [_P, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P]
+    for name in ("sf_checkpoint_save", "sf_checkpoint_restore"):
+        getattr(L, name).argtypes = [ctypes.POINTER(sf_matrix), ctypes.POINTER(sf_checkpoint), ctypes.c_int, _P, _P]
+        getattr(L, name).restype = ctypes.c_int
     for name in ("sf_mask_init", "sf_mask_update", "sf_masked_dw", "sf_embed_grad", "sf_adam_tables",
                  "sf_sparse_update", "sf_quantize_init"):
         getattr(L, name).restype = ctypes.c_int
@@ -310,3 +318,39 @@ def sf_quantize_init(W, mat: Matrix, stream=None):
 
 def sf_version() -> int:
     return load().sf_version()
+
+
+class Checkpoint:
+    """Device buffers of an active-row checkpoint of one matrix (section 2.6)."""
+
+    def __init__(self, cap: int, C: int, device="cuda"):
+        self.cap, self.C = cap, C
+        n = max(cap, 1)
+        self.count = torch.zeros(1, dtype=torch.int32, device=device)
+        self.rows = torch.zeros(n, dtype=torch.int32, device=device)
+        self.q = torch.zeros((n, C), dtype=torch.int8, device=device)
+        self.s = torch.zeros(n, dtype=torch.float32, device=device)
+        self.delta = torch.zeros((n, C), dtype=torch.float32, device=device)
+        self.m = torch.zeros((n, C), dtype=torch.int16, device=device)
+        self.v = torch.zeros((n, C), dtype=torch.int16, device=device)
+        self.step = torch.zeros(n, dtype=torch.int32, device=device)
+
+    def struct(self) -> sf_checkpoint:
+        return sf_checkpoint(self.cap, _ptr(self.count), _ptr(self.rows), _ptr(self.q), _ptr(self.s),
+                             _ptr(self.delta), _ptr(self.m), _ptr(self.v), _ptr(self.step))
+
+
+def _ckpt_call(name, mats, ckpts, status, stream):
+    n = len(mats)
+    arr = (sf_matrix * n)(*mats)
+    carr = (sf_checkpoint * n)(*[c.struct() for c in ckpts])
+    _check(getattr(load(), name)(arr, carr, n, _ptr(status), _stream(stream)), name)
+
+
+def sf_checkpoint_save(mats, ckpts, status=None, stream=None):
+    """mats: list of sf_matrix (matrix_struct); ckpts: list of Checkpoint, same order."""
+    _ckpt_call("sf_checkpoint_save", mats, ckpts, status, stream)
+
+
+def sf_checkpoint_restore(mats, ckpts, status=None, stream=None):
+    _ckpt_call("sf_checkpoint_restore", mats, ckpts, status, stream)

@@ -72,6 +72,10 @@ def _declare(L):
     L.orc_quantize_rows.argtypes = [_I, _I, _P, _P, _P, _P]
     L.orc_rebuild_rows.restype = None
     L.orc_rebuild_rows.argtypes = [_I, _I, _P, _P, _P, _P]
+    L.orc_checkpoint_save.restype = _I
+    L.orc_checkpoint_save.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P]
+    L.orc_checkpoint_restore.restype = None
+    L.orc_checkpoint_restore.argtypes = [_I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P]
     L.orc_bias_correction.restype = _F
     L.orc_bias_correction.argtypes = [_F, _I]
     L.orc_update.restype = None
@@ -270,3 +274,30 @@ def update(a: MatrixState, g: np.ndarray, hp: AdamHP, partner: MatrixState | Non
                      None if partner is None else _ptr(pg),
                      float(c_self), float(c_partner), hp.lr, hp.beta1, hp.beta2,
                      hp.one_minus_b1, hp.one_minus_b2, hp.eps, hp.wd, hp.clip, _ptr(scratch))
+
+
+# ---- section 2.6: checkpoint and rewind of the active rows ----------------------------------
+
+class Checkpoint:
+    """Snapshot of a MatrixState's active rows (row ids, q, s, delta, m, v, step)."""
+
+    def __init__(self, st: MatrixState, cap: int | None = None):
+        cap = st.R if cap is None else cap
+        C = st.C
+        self.rows = np.zeros(cap, np.int32)
+        self.q = np.zeros((cap, C), np.int8)
+        self.s = np.zeros(cap, np.float32)
+        self.delta = np.zeros((cap, C), np.float32)
+        self.m = np.zeros((cap, C), np.uint16)
+        self.v = np.zeros((cap, C), np.uint16)
+        self.step = np.zeros(cap, np.int32)
+        self.n = lib().orc_checkpoint_save(
+            st.R, C, _ptr(st.q), _ptr(st.s), _ptr(st.delta), _ptr(st.m), _ptr(st.v), _ptr(st.step),
+            _ptr(st.words), cap, _ptr(self.rows), _ptr(self.q), _ptr(self.s), _ptr(self.delta),
+            _ptr(self.m), _ptr(self.v), _ptr(self.step))
+
+    def restore(self, st: MatrixState):
+        lib().orc_checkpoint_restore(
+            st.R, st.C, _ptr(st.q), _ptr(st.s), _ptr(st.delta), _ptr(st.m), _ptr(st.v), _ptr(st.step),
+            _ptr(st.live), _ptr(st.words), self.n, _ptr(self.rows), _ptr(self.q), _ptr(self.s),
+            _ptr(self.delta), _ptr(self.m), _ptr(self.v), _ptr(self.step))

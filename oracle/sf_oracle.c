@@ -399,3 +399,71 @@ void orc_rebuild_rows(int R, int C, const int8_t *q, const float *s, const float
             W[i] = fmaf(s[r], (float)q[i], delta[i]);
         }
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* 2.6 Checkpoint and rewind of the active rows.                                               */
+/* ------------------------------------------------------------------------------------------ */
+
+/*
+ * Section 2.6 keeps a checkpoint of the active rows only. Reading taken: a checkpoint is a
+ * snapshot, at save time, of every active row's storage and optimizer state: its row id, q, s,
+ * delta, m, v and step count. Rows are saved in ascending row order. Returns the rows saved.
+ * Buffers hold cap rows (rows beyond cap are not saved; the return value says how many were).
+ */
+int orc_checkpoint_save(int R, int C, const int8_t *q, const float *s, const float *delta,
+                        const uint16_t *m, const uint16_t *v, const int32_t *step,
+                        const uint32_t *words, int cap, int32_t *rows, int8_t *cq, float *cs,
+                        float *cdelta, uint16_t *cm, uint16_t *cv, int32_t *cstep)
+{
+    int k = 0;
+    for (int r = 0; r < R; ++r) {
+        if (!((words[r / 32] >> (r % 32)) & 1))
+            continue;
+        if (k >= cap)
+            return k;
+        rows[k] = r;
+        cs[k] = s[r];
+        cstep[k] = step[r];
+        for (int c = 0; c < C; ++c) {
+            size_t i = (size_t)r * C + c, j = (size_t)k * C + c;
+            cq[j] = q[i];
+            cdelta[j] = delta[i];
+            cm[j] = m[i];
+            cv[j] = v[i];
+        }
+        ++k;
+    }
+    return k;
+}
+
+/*
+ * Rewind: every saved row gets back its q, s and delta, and its live weights are rebuilt from
+ * them (bf16 of fma(s, q, delta)). Moments exist only for active rows (section 2.3), so a saved
+ * row gets its moments and step count back only if it is active now; otherwise they stay
+ * dropped. Rows that were not saved are left as they are.
+ */
+void orc_checkpoint_restore(int R, int C, int8_t *q, float *s, float *delta, uint16_t *m,
+                            uint16_t *v, int32_t *step, uint16_t *live, const uint32_t *words,
+                            int n, const int32_t *rows, const int8_t *cq, const float *cs,
+                            const float *cdelta, const uint16_t *cm, const uint16_t *cv,
+                            const int32_t *cstep)
+{
+    (void)R;
+    for (int k = 0; k < n; ++k) {
+        int r = rows[k];
+        int active = (words[r / 32] >> (r % 32)) & 1;
+        s[r] = cs[k];
+        if (active)
+            step[r] = cstep[k];
+        for (int c = 0; c < C; ++c) {
+            size_t i = (size_t)r * C + c, j = (size_t)k * C + c;
+            q[i] = cq[j];
+            delta[i] = cdelta[j];
+            live[i] = orc_f32_to_bf16(fmaf(cs[k], (float)cq[j], cdelta[j]));
+            if (active) {
+                m[i] = cm[j];
+                v[i] = cv[j];
+            }
+        }
+    }
+}

@@ -67,7 +67,8 @@ def _c_struct_fields(name):
     return fields
 
 
-@pytest.mark.parametrize("name", ["sf_mask", "sf_mask_src", "sf_dw_problem", "sf_matrix", "sf_adam"])
+@pytest.mark.parametrize("name", ["sf_mask", "sf_mask_src", "sf_dw_problem", "sf_matrix", "sf_adam",
+                                  "sf_checkpoint"])
 def test_binding_structs_follow_the_header(name):
     py = [f[0] for f in getattr(binding, name)._fields_]
     assert py == _c_struct_fields(name)

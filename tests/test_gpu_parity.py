@@ -562,3 +562,101 @@ def test_update_flags_nonfinite_gradients_and_fp16_overflow(sf):
         sf.sf_sparse_update([sf.matrix_struct(mat)], hp, status)
         flagged = bool(int(host(status)[0]) & sf.SF_STATUS_NONFINITE)
         assert flagged == (case != "clean"), case
+
+
+# =============================================================================================
+# section 2.6: checkpoint and rewind of the active rows
+# =============================================================================================
+
+def _compare_checkpoint(ck, oc: "orc.Checkpoint"):
+    n = int(host(ck.count)[0])
+    assert n == oc.n
+    assert np.array_equal(host(ck.rows)[:n], oc.rows[:n])
+    assert host(ck.q)[:n].tobytes() == oc.q[:n].tobytes()
+    assert host(ck.s)[:n].tobytes() == oc.s[:n].tobytes()
+    assert host(ck.delta)[:n].tobytes() == oc.delta[:n].tobytes()
+    assert np.array_equal(host(ck.m).view(np.uint16)[:n], oc.m[:n])
+    assert np.array_equal(host(ck.v).view(np.uint16)[:n], oc.v[:n])
+    assert np.array_equal(host(ck.step)[:n], oc.step[:n])
+
+
+def test_checkpoint_save_train_restore_matches_oracle(sf):
+    # Three matrices (one 11008 wide, one paired couple): two steps, save, two more steps with
+    # changed masks (some saved rows drop out, new rows come in), restore, one more step.
+    shapes = [(128, 272), (128, 272), (64, 11008)]
+    pairs = {0: 1, 1: 0, 2: -1}
+    hp, ohp = sf.AdamParams(lr=2e-3), orc.AdamHP(lr=2e-3)
+    sts = [orc.MatrixState(synth.weights_f32(synth.rng(31, "weights", i), R, C))
+           for i, (R, C) in enumerate(shapes)]
+    mats = [_state_from_oracle(sf, s_, R) for s_, (R, _) in zip(sts, shapes)]
+    g = synth.rng(31, "rows")
+    status = sf.status_word()
+    cks = [sf.Checkpoint(R, C, DEV) for R, C in shapes]
+    saved_rows = None
+
+    def step(k):
+        grads = [_grad_rows(31, 10 * k + i, R, C) for i, (R, C) in enumerate(shapes)]
+        for m_, gr in zip(mats, grads):
+            _load_grad(m_, gr)
+        sf.sf_sparse_update([sf.matrix_struct(mats[i], pairs[i], 1.0, 0.5 if pairs[i] >= 0 else 0.0)
+                             for i in range(3)], hp, status)
+        for i in range(3):
+            p = pairs[i]
+            if p >= 0:
+                orc.update(sts[i], grads[i], ohp, partner=sts[p], pg=grads[p], c_self=1.0, c_partner=0.5)
+            else:
+                orc.update(sts[i], grads[i], ohp)
+
+    for k in range(5):
+        if k == 2:
+            sf.sf_checkpoint_save([sf.matrix_struct(m_) for m_ in mats], cks, status)
+            ocks = [orc.Checkpoint(s_) for s_ in sts]
+            for ck, oc in zip(cks, ocks):
+                _compare_checkpoint(ck, oc)
+            saved_rows = [oc.rows[:oc.n].copy() for oc in ocks]
+        if k in (0, 3):
+            words = [synth.words_from_rows(R, np.sort(g.choice(R, R // 4, replace=False)))
+                     for R, _ in shapes]
+            if k == 3:                                   # keep half of the saved rows active
+                for i, (R, _) in enumerate(shapes):
+                    keep = saved_rows[i][::2]
+                    words[i] = synth.words_from_rows(R, np.union1d(keep, synth.rows_from_words(words[i])))
+            for st_, w in zip(sts, words):
+                st_.set_mask(w)
+            _set_words(sf, list(zip(mats, words)))
+        if k == 4:
+            sf.sf_checkpoint_restore([sf.matrix_struct(m_) for m_ in mats], cks, status)
+            for s_, oc in zip(sts, ocks):
+                oc.restore(s_)
+            for m_, s_, rows in zip(mats, sts, saved_rows):
+                _compare_matrix(m_, s_)
+                assert np.array_equal(host(m_.live).view(np.uint16)[rows], s_.live[rows])
+        step(k)
+        for m_, s_ in zip(mats, sts):
+            _compare_matrix(m_, s_)
+    assert host(status)[0] == 0
+
+
+def test_checkpoint_capacity_overflow_and_arguments(sf):
+    R, C = 64, 32
+    st = orc.MatrixState(synth.weights_f32(synth.rng(32, "weights"), R, C))
+    words = synth.words_from_rows(R, [3, 7, 40, 41, 60])
+    st.set_mask(words)
+    mat = _state_from_oracle(sf, st, R)
+    _set_words(sf, [(mat, words)])
+    status = sf.status_word()
+    ck = sf.Checkpoint(3, C, DEV)
+    sf.sf_checkpoint_save([sf.matrix_struct(mat)], [ck], status)
+    _compare_checkpoint(ck, orc.Checkpoint(st, cap=3))
+    assert int(host(status)[0]) == sf.SF_STATUS_SLOT_OVERFLOW
+    # an empty checkpoint restores nothing
+    q0 = host(mat.q).copy()
+    empty = sf.Checkpoint(0, C, DEV)
+    sf.sf_checkpoint_save([sf.matrix_struct(mat)], [empty])
+    sf.sf_checkpoint_restore([sf.matrix_struct(mat)], [empty])
+    assert host(mat.q).tobytes() == q0.tobytes()
+    # C not a multiple of 16
+    bad = sf.Matrix(64, 24, 8, DEV)
+    sf.sf_mask_init(bad.mask)
+    with pytest.raises(RuntimeError):
+        sf.sf_checkpoint_save([sf.matrix_struct(bad)], [sf.Checkpoint(4, 24, DEV)])

@@ -50,6 +50,13 @@ MUTANTS = {
                            "if (drop >= 0x8000u)"),
     "moments_kept_on_deactivation": ("if (was == now)\n            continue;",
                                      "if (was == now || was)\n            continue;"),
+    "restore_forgets_scale": ("        s[r] = cs[k];\n", "\n"),
+    "restore_moments_to_inactive_rows": ("            if (active) {\n                m[i] = cm[j];",
+                                         "            if (1) {\n                m[i] = cm[j];"),
+    "restore_live_not_rebuilt": ("live[i] = orc_f32_to_bf16(fmaf(cs[k], (float)cq[j], cdelta[j]));",
+                                 "(void)live;"),
+    "restore_live_without_residual": ("live[i] = orc_f32_to_bf16(fmaf(cs[k], (float)cq[j], cdelta[j]));",
+                                      "live[i] = orc_f32_to_bf16(cs[k] * (float)cq[j]);"),
 }
 
 PIN_TESTS = [f for name, f in inspect.getmembers(pins, inspect.isfunction)

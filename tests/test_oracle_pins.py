@@ -537,3 +537,48 @@ def test_reactivated_row_restarts_from_zero_moments():
     orc.update(st, gr, HP)
     expect = W[3].astype(np.float64) - HP.lr * gr[3] / (np.abs(gr[3]) + HP.eps)
     assert np.all(np.abs(st.weight()[3] - expect) <= 2 * np.spacing(np.abs(expect).astype(np.float32)))
+
+
+# =============================================================================================
+# Section 2.6: checkpoint and rewind of the active rows
+# =============================================================================================
+
+def test_checkpoint_round_trip_restores_saved_rows_only():
+    # Save after two steps; train on with a changed mask (a saved row turns inactive, a new row
+    # turns active); restore. Saved rows get back exactly their saved storage, their live row is
+    # bf16 of the restored weight, moments come back only where the row is active now; rows not
+    # in the checkpoint keep whatever they had.
+    g = np.random.default_rng(21)
+    R, C = 64, 48
+    st = orc.MatrixState(synth.weights_f32(g, R, C))
+    st.set_mask(synth.words_from_rows(R, [2, 9, 40, 41]))
+    for _ in range(2):
+        orc.update(st, _grad(g, R, C), HP)
+    saved = {k: getattr(st, k).copy() for k in ("q", "s", "delta", "m", "v", "step")}
+    ck = orc.Checkpoint(st)
+    assert ck.n == 4 and list(ck.rows[:4]) == [2, 9, 40, 41]
+    st.set_mask(synth.words_from_rows(R, [2, 9, 41, 50]))          # row 40 out, row 50 in
+    for _ in range(3):
+        orc.update(st, _grad(g, R, C), HP)
+    before = {k: getattr(st, k).copy() for k in ("q", "s", "delta", "m", "v", "step", "live")}
+    ck.restore(st)
+    for r in (2, 9, 40, 41):
+        assert st.q[r].tobytes() == saved["q"][r].tobytes()
+        assert st.s[r] == saved["s"][r] and st.delta[r].tobytes() == saved["delta"][r].tobytes()
+        expect_live = synth.f32_to_bf16_bits(orc.rebuild(saved["q"][r:r + 1], saved["s"][r:r + 1],
+                                                         saved["delta"][r:r + 1]))[0]
+        assert np.array_equal(st.live[r], expect_live)
+    for r in (2, 9, 41):                                              # still active: moments back
+        assert st.m[r].tobytes() == saved["m"][r].tobytes() and st.step[r] == saved["step"][r]
+    assert not st.m[40].any() and st.step[40] == 0                    # inactive now: stay dropped
+    for k in ("q", "s", "delta", "m", "v", "step", "live"):           # row 50 was not saved
+        assert getattr(st, k)[50].tobytes() == before[k][50].tobytes()
+
+
+def test_checkpoint_capacity_keeps_the_first_rows():
+    g = np.random.default_rng(22)
+    R, C = 64, 16
+    st = orc.MatrixState(synth.weights_f32(g, R, C))
+    st.set_mask(synth.words_from_rows(R, [1, 5, 33, 60]))
+    ck = orc.Checkpoint(st, cap=2)
+    assert ck.n == 2 and list(ck.rows[:2]) == [1, 5]
