@@ -22,6 +22,7 @@ from . import binding as sf
 LLAMA_7B_LAYER = (("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
                   ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008))
 PARTNER = {"q": "o", "o": "q", "k": "v", "v": "k", "gate": "up", "up": "gate"}
+PAIR_OF = {"q": "q-o", "o": "q-o", "k": "k-v", "v": "k-v", "gate": "gate-up", "up": "gate-up"}
 # coupling strength of each pair (section 2.4): strong for gate-up, weaker for attention pairs
 STRENGTH = {"gate": 0.6, "up": 0.6, "q": 0.4, "o": 0.4, "k": 0.4, "v": 0.4}
 # which layer input each projection reads: attention input, attention output, FFN input, FFN mid
@@ -181,6 +182,15 @@ class StepPlan:
         c = math.cos(math.radians(phase_deg))
         for i, p in enumerate(self.model.projs):
             self.upd_arr[i + off].c_partner = STRENGTH.get(p.name, 0.0) * c
+
+    def set_mix(self, c_self: float, c_partner: dict):
+        """Per-pair coefficients from a schedule (helix.Helix.coefficients): c_partner maps a
+        pair name ("q-o", "k-v", "gate-up") to the weight of the partner's gradient."""
+        off = 1 if self.model.emb is not None else 0
+        for i, p in enumerate(self.model.projs):
+            pair = PAIR_OF.get(p.name)
+            self.upd_arr[i + off].c_self = c_self
+            self.upd_arr[i + off].c_partner = c_partner.get(pair, 0.0) if pair else 0.0
 
     # the four calls of one step --------------------------------------------------------------
     def masks(self, status, stream):
