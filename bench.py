@@ -38,6 +38,7 @@ TRAFFIC_PER_LAYER = {"masks": (348.56e6 + 3.85e6 + 1.08e6) / 2,
                      "masked_dw": (203.92e6 + 8.32e6 + 173.74e6 + 3.98e6) / 2}
 UNIT = "active-row updates/s"
 SEED = 3
+SWEEP_SEED = 4
 
 
 def parse():
@@ -52,6 +53,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps (capped at 20)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="density sweep of one 11008 x 4096 projection (T = 4096), scattered and "
+                         "clustered rows, with a dense bf16 GEMM and a fused dense Adam as context; "
+                         "prints one JSON line per point (not the headline metric)")
     return ap.parse_args()
 
 
@@ -322,10 +327,134 @@ def run_reference(args):
     return 0
 
 
+SWEEP_DENSITIES = (0.001, 0.005, 0.01, 0.05, 0.2, 0.5)
+
+
+def run_sweep(args):
+    """One projection (R = 11008, C = 4096, T = 4096) at several active-row densities: masks from
+    the row tracker, masked dW, fused update; each stage timed with CUDA events on the launching
+    stream. Context lines: the dense dW as one cuBLAS bf16 GEMM (torch.matmul) and one dense
+    fused Adam step (torch.optim.Adam, fused) over the same fp32 matrix."""
+    import torch
+    from masked_optimizer_step_b200 import binding as sf
+    from masked_optimizer_step_b200 import synth
+    sf.load()
+    device = "cuda:0"
+    torch.cuda.set_device(0)
+    R, C, T = 11008, 4096, 4096
+    steps, warm = max(args.steps, 3), max(args.warmup, 3)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    tf_sus = float(peaks.get("bf16_tflops_sustained", 1400.0))
+    stream = torch.cuda.current_stream()
+    A = synth.device_normal_bf16((T, C), SWEEP_SEED, "act", device=device)
+    dX = synth.device_normal_bf16((T, R), SWEEP_SEED, "dx", device=device)
+    W0 = synth.device_weights_f32(R, C, SWEEP_SEED, 0, device=device)
+    hp = sf.AdamParams(device=device)
+    status = sf.status_word(device)
+    lines = []
+    for kind in ("scattered", "clustered"):
+        for d in SWEEP_DENSITIES:
+            g = synth.rng(SWEEP_SEED, "rows", int(d * 1e4), int(kind == "clustered"))
+            rows = synth.scattered_rows(g, R, d) if kind == "scattered" else synth.clustered_rows(g, R, d)
+            cap = min(R, -(-len(rows) // 32) * 32 + 32)
+            gain = torch.from_numpy(synth.tracker_gains(R, rows)).to(device)
+            gen = synth.device_generator(SWEEP_SEED, "tracker", int(d * 1e4), device=device)
+            Y = torch.randn((T, R), generator=gen, device=device).mul_(gain[None, :]).to(torch.bfloat16)
+            mat = sf.Matrix(R, C, cap, device)
+            sf.sf_mask_init(mat.mask)
+            sf.sf_quantize_init(W0, mat)
+            srcs = [sf.make_src(sf.SF_SRC_OUTPUT_BF16, Y, n=T, ld=Y.stride(0))]
+            probs = [sf.dw_problem(dX, A, mat.mask, mat.grad)]
+            ws = sf.dw_workspace(probs, device)
+            ms_struct = [sf.matrix_struct(mat)]
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+            for k in range(warm + steps):
+                e = ev[k - warm] if k >= warm else None
+                if e:
+                    e[0].record(stream)
+                sf.sf_mask_update([mat.mask], srcs, 0.01, status, stream)
+                if e:
+                    e[1].record(stream)
+                sf.sf_masked_dw(probs, status, stream, ws)
+                if e:
+                    e[2].record(stream)
+                sf.sf_sparse_update(ms_struct, hp, status, stream)
+                if e:
+                    e[3].record(stream)
+            torch.cuda.synchronize()
+            st = np.zeros(3)
+            for e in ev:
+                for j in range(3):
+                    st[j] += e[j].elapsed_time(e[j + 1])
+            st /= steps
+            cnt = mat.mask.counts.cpu().numpy()
+            n_rows, n_tiles = int(cnt[0]), int(cnt[1])
+            mt_tiles = (n_tiles + 3) // 4
+            rows_mode = n_rows <= -(-cap // 32) * 32 and -(-n_rows // 128) < mt_tiles
+            mt = -(-n_rows // 128) if rows_mode else mt_tiles
+            dw_exec = mt * 128 * C * T * 2
+            dw_useful = n_rows * C * T * 2
+            dw_bytes = T * C * 2 + n_rows * C * 4 + (T * n_rows * 2 if rows_mode else n_tiles * 32 * T * 2)
+            upd_bytes = n_rows * C * 24 + n_rows * 8
+            line = {"workload": "density sweep, one 11008x4096 projection, T=4096", "masks": kind,
+                    "density_requested": d, "active_rows": n_rows, "active_tile_frac": n_tiles / (R // 32),
+                    "dw_mode": "rows" if rows_mode else "tiles",
+                    "ms": {"masks": st[0], "masked_dw": st[1], "sparse_update": st[2], "step": float(st.sum())},
+                    "masked_dw_tflops_useful": dw_useful / (st[1] / 1e3) / 1e12,
+                    "masked_dw_tflops_executed": dw_exec / (st[1] / 1e3) / 1e12,
+                    "masked_dw_gbs": dw_bytes / (st[1] / 1e3) / 1e9,
+                    "update_gbs": upd_bytes / (st[2] / 1e3) / 1e9,
+                    "update_frac_hbm": upd_bytes / (st[2] / 1e3) / 1e9 / hbm,
+                    "tracker_gbs": T * R * 2 / (st[0] / 1e3) / 1e9,
+                    "device_status": int(status.cpu()[0])}
+            lines.append(line)
+            print(json.dumps(line), flush=True)
+            del mat, Y, probs, ws, srcs
+            torch.cuda.empty_cache()
+    # dense context: dW = dX^T A as one bf16 GEMM, and one fused Adam step on an fp32 matrix
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for _ in range(warm):
+        torch.matmul(dX.t(), A)
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(steps):
+        torch.matmul(dX.t(), A)
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    gemm_ms = ev[0].elapsed_time(ev[1]) / steps
+    param = torch.nn.Parameter(W0.clone())
+    param.grad = torch.randn_like(param)
+    opt = torch.optim.Adam([param], lr=1e-4, fused=True)
+    for _ in range(warm):
+        opt.step()
+    torch.cuda.synchronize()
+    ev[0].record(stream)
+    for _ in range(steps):
+        opt.step()
+    ev[1].record(stream)
+    torch.cuda.synchronize()
+    adam_ms = ev[0].elapsed_time(ev[1]) / steps
+    dense = {"workload": "dense context, one 11008x4096 projection, T=4096",
+             "dense_dw_gemm_ms": gemm_ms, "dense_dw_output": "bf16 (torch.matmul of bf16 operands)", "dense_dw_tflops": 2 * T * R * C / (gemm_ms / 1e3) / 1e12,
+             "dense_adam_fused_ms": adam_ms,
+             "dense_adam_gbs": R * C * 28 / (adam_ms / 1e3) / 1e9,
+             "dense_step_ms": gemm_ms + adam_ms,
+             "peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": tf_sus}}
+    print(json.dumps(dense), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
     rank, world, local = dist_env()
     import torch
     import torch.distributed as dist

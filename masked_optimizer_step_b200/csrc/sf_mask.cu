@@ -25,9 +25,10 @@ constexpr int kAccumThreads = 256;
 constexpr int kColsPerThread = 8;                            // one 16-byte load of bf16
 constexpr int kColsPerCta = kAccumThreads * kColsPerThread;  // 2048
 constexpr int kTokensPerSeg = 512;
+constexpr int kMinTokensPerSeg = 32;
 constexpr int kTokensPerTokCta = kAccumThreads * 8;          // histogram: 8 ids per thread
 constexpr int kFinalizeThreads = 1024;
-constexpr int kMaxRows = 262144;                             // words of two masks fit in smem
+constexpr int kMaxRows = 262144;                             // three bit masks per tile fit in smem
 
 struct MaskDesc {
     int32_t R, slot_cap, kind, n;
@@ -138,159 +139,177 @@ mask_accum_kernel(const __grid_constant__ MaskBatch b, uint32_t *status)
     if (nonfinite) set_status(status, SF_STATUS_NONFINITE);
 }
 
+// Finalize, one CTA per mask. Phase 2 runs one warp per 32-row tile (lane = row) and issues the
+// loads of kBatch tiles before using any of them, so a warp has several independent DRAM round
+// trips in flight; the new, released and needing-a-slot bit masks of every tile stay in shared
+// memory. The slot sweeps and the lists then go over rounds of kRound words: a block scan of the
+// per-word counts gives every tile its offsets, and a warp per tile writes its rows' entries,
+// touching global memory only for rows that change state.
+constexpr int kBatch = 8;
+constexpr int kRound = 512;       // words per scan round; per-round sums stay below 2^15 per field
+
 __global__ void __launch_bounds__(kFinalizeThreads)
 mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *status)
 {
     extern __shared__ uint32_t smem_words[];
     __shared__ int scan_scratch[33];
     __shared__ uint32_t max_scratch[33];
-    __shared__ int s_free_top, s_rows, s_tiles, s_fresh;
+    __shared__ int s_off[kRound];
+    __shared__ int s_toff[kRound];
 
     const MaskDesc &d = b.d[blockIdx.x];
     const int R = d.R, nw = R >> 5;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nwarps = blockDim.x >> 5;
+    constexpr int nwarps = kFinalizeThreads / 32;
+    const uint32_t lt = (1u << lane) - 1u;
     uint32_t *new_w = smem_words;
-    uint32_t *old_w = smem_words + nw;
+    uint32_t *rel_w = smem_words + nw;
+    uint32_t *need_w = smem_words + 2 * nw;
+    const int kind = d.kind;
+    const uint32_t *src_u32 = static_cast<const uint32_t *>(d.src);
 
     // (1) busiest row of the window
     uint32_t hmax = 0;
-    if (d.kind == SF_SRC_TOKENS || d.kind == SF_SRC_OUTPUT_BF16) {
-        for (int r = tid; r < R; r += blockDim.x) hmax = max(hmax, d.accum[r]);
-    } else if (d.kind == SF_SRC_HITS_U32) {
-        const uint32_t *hits = static_cast<const uint32_t *>(d.src);
-        for (int r = tid; r < R; r += blockDim.x) hmax = max(hmax, hits[r]);
+    if (kind == SF_SRC_TOKENS || kind == SF_SRC_OUTPUT_BF16) {
+#pragma unroll 4
+        for (int r = tid; r < R; r += kFinalizeThreads) hmax = max(hmax, d.accum[r]);
+    } else if (kind == SF_SRC_HITS_U32) {
+#pragma unroll 4
+        for (int r = tid; r < R; r += kFinalizeThreads) hmax = max(hmax, src_u32[r]);
     }
     hmax = block_max_u32(hmax, max_scratch);
+    const float H = kind == SF_SRC_OUTPUT_BF16 ? __uint_as_float(hmax) : __uint2float_rn(hmax);
 
-    // (2) charge rule and new mask words: one warp per 32-row tile
-    for (int w = warp; w < nw; w += nwarps) {
-        const int r = (w << 5) + lane;
-        bool act;
-        if (d.kind == SF_SRC_WORDS) {
-            act = (static_cast<const uint32_t *>(d.src)[w] >> lane) & 1u;
-        } else {
-            float h, H;
-            if (d.kind == SF_SRC_TOKENS) {
-                h = __uint2float_rn(d.accum[r]);
-                H = __uint2float_rn(hmax);
-                d.accum[r] = 0u;                       // ready for the next window
-            } else if (d.kind == SF_SRC_OUTPUT_BF16) {
-                h = __uint_as_float(d.accum[r]);
-                H = __uint_as_float(hmax);
-                d.accum[r] = 0u;
-            } else {
-                h = __uint2float_rn(static_cast<const uint32_t *>(d.src)[r]);
-                H = __uint2float_rn(hmax);
+    // (2) charge rule, new mask word, and which rows release or need a slot
+    for (int w0 = warp; w0 < nw; w0 += nwarps * kBatch) {
+        uint32_t hv[kBatch], ow[kBatch];
+        float qv[kBatch];
+        int sl[kBatch];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const int w = w0 + k * nwarps;
+            hv[k] = 0u;
+            ow[k] = 0u;
+            qv[k] = 0.0f;
+            sl[k] = -1;
+            if (w < nw) {
+                const int r = (w << 5) + lane;
+                if (kind == SF_SRC_WORDS) {
+                    hv[k] = src_u32[w];
+                } else {
+                    hv[k] = kind == SF_SRC_HITS_U32 ? src_u32[r] : d.accum[r];
+                    qv[k] = d.charge[r];
+                }
+                ow[k] = d.words[w];
+                sl[k] = d.row_slot[r];
             }
-            const float share = (H == 0.0f) ? 0.0f : __fdiv_rn(h, H);
-            const float q = __fadd_rn(__fmul_rn(0.5f, d.charge[r]), __fmul_rn(0.5f, share));
-            d.charge[r] = q;
-            act = q >= thr;
         }
-        const uint32_t word = __ballot_sync(0xffffffffu, act);
-        if (lane == 0) {
-            new_w[w] = word;
-            old_w[w] = d.words[w];
+#pragma unroll
+        for (int k = 0; k < kBatch; ++k) {
+            const int w = w0 + k * nwarps;
+            if (w >= nw) break;                                  // uniform across the warp
+            const int r = (w << 5) + lane;
+            bool act;
+            if (kind == SF_SRC_WORDS) {
+                act = (hv[k] >> lane) & 1u;
+            } else {
+                const float h = kind == SF_SRC_OUTPUT_BF16 ? __uint_as_float(hv[k]) : __uint2float_rn(hv[k]);
+                const float share = (H == 0.0f) ? 0.0f : __fdiv_rn(h, H);
+                const float q = __fadd_rn(__fmul_rn(0.5f, qv[k]), __fmul_rn(0.5f, share));
+                d.charge[r] = q;
+                if (kind != SF_SRC_HITS_U32) d.accum[r] = 0u;      // ready for the next window
+                act = q >= thr;
+            }
+            const bool was = (ow[k] >> lane) & 1u;
+            const uint32_t nword = __ballot_sync(0xffffffffu, act);
+            const uint32_t rel = __ballot_sync(0xffffffffu, was && !act && sl[k] >= 0);
+            const uint32_t need = __ballot_sync(0xffffffffu, act && sl[k] < 0);
+            if (lane == 0) {
+                new_w[w] = nword;
+                rel_w[w] = rel;
+                need_w[w] = need;
+            }
         }
-    }
-    if (tid == 0) {
-        s_free_top = d.counts[2];
-        s_rows = 0;
-        s_tiles = 0;
-        s_fresh = 0;
     }
     __syncthreads();
 
-    // (3) rows that turned inactive return their slots, ascending row order
-    for (int base = 0; base < nw; base += blockDim.x) {
+    // (3) rows that turned inactive push their slots onto the free stack, ascending row order
+    int top = d.counts[2];
+    for (int base = 0; base < nw; base += kRound) {
         const int w = base + tid;
-        const uint32_t gone = (w < nw) ? (old_w[w] & ~new_w[w]) : 0u;
-        int mine = 0;
-        for (uint32_t bits = gone; bits; bits &= bits - 1)
-            mine += d.row_slot[(w << 5) + __ffs(bits) - 1] >= 0;
+        const int c = (tid < kRound && w < nw) ? __popc(rel_w[w]) : 0;
         int total;
-        const int off = block_exclusive_scan(mine, scan_scratch, &total);
-        const int top = s_free_top;
-        int j = 0;
-        for (uint32_t bits = gone; bits; bits &= bits - 1) {
-            const int r = (w << 5) + __ffs(bits) - 1;
-            const int s = d.row_slot[r];
-            if (s >= 0) {
-                d.free_slots[top + off + j] = s;
-                ++j;
-                d.row_slot[r] = -1;
+        const int off = block_exclusive_scan(c, scan_scratch, &total);
+        if (tid < kRound) s_off[tid] = off;
+        __syncthreads();
+        if (total) {
+            for (int j = warp; j < kRound && base + j < nw; j += nwarps) {
+                const uint32_t rel = rel_w[base + j];
+                if ((rel >> lane) & 1u) {
+                    const int r = ((base + j) << 5) + lane;
+                    d.free_slots[top + s_off[j] + __popc(rel & lt)] = d.row_slot[r];
+                    d.row_slot[r] = -1;
+                }
             }
         }
-        __syncthreads();
-        if (tid == 0) s_free_top = top + total;
+        top += total;
         __syncthreads();
     }
 
-    // (4) active rows without a slot take one from the top of the stack, ascending row order
-    int over = 0;
-    for (int base = 0; base < nw; base += blockDim.x) {
+    // (4) rows that need a slot pop one from the top (ascending row order); lists and words
+    const int top2 = top;
+    int need_base = 0, rows_base = 0, tiles_base = 0, over = 0;
+    for (int base = 0; base < nw; base += kRound) {
         const int w = base + tid;
-        const uint32_t act = (w < nw) ? new_w[w] : 0u;
-        int mine = 0;
-        for (uint32_t bits = act; bits; bits &= bits - 1)
-            mine += d.row_slot[(w << 5) + __ffs(bits) - 1] < 0;
-        int total;
-        const int off = block_exclusive_scan(mine, scan_scratch, &total);
-        const int top = s_free_top;
-        int j = 0;
-        for (uint32_t bits = act; bits; bits &= bits - 1) {
-            const int r = (w << 5) + __ffs(bits) - 1;
-            if (d.row_slot[r] >= 0) continue;
-            const int idx = off + j;
-            ++j;
-            if (idx < top) {
-                const int s = d.free_slots[top - 1 - idx];
-                d.row_slot[r] = s;
-                d.slot_step[s] = 0;                    // fresh moments
-            } else {
-                ++over;
+        const bool mine = tid < kRound && w < nw;
+        const uint32_t word = mine ? new_w[w] : 0u;
+        const uint32_t nd = mine ? need_w[w] : 0u;
+        int tot1, tot2;
+        const int off1 = block_exclusive_scan((__popc(nd) << 16) | __popc(word), scan_scratch, &tot1);
+        const int off2 = block_exclusive_scan(word != 0u, scan_scratch, &tot2);
+        if (tid < kRound) {
+            s_off[tid] = off1;
+            s_toff[tid] = off2;
+        }
+        __syncthreads();
+        for (int j = warp; j < kRound && base + j < nw; j += nwarps) {
+            const int wj = base + j;
+            const uint32_t wd = new_w[wj], ndw = need_w[wj];
+            const int r = (wj << 5) + lane;
+            const int roff = rows_base + (s_off[j] & 0xFFFF);
+            if ((ndw >> lane) & 1u) {
+                const int idx = need_base + (s_off[j] >> 16) + __popc(ndw & lt);
+                if (idx < top2) {
+                    const int sl = d.free_slots[top2 - 1 - idx];
+                    d.row_slot[r] = sl;
+                    d.slot_step[sl] = 0;                           // fresh moments
+                } else {
+                    ++over;
+                }
+            }
+            if ((wd >> lane) & 1u) d.active_rows[roff + __popc(wd & lt)] = r;
+            if (lane == 0) {
+                d.words[wj] = wd;
+                if (wd) {
+                    const int t = tiles_base + s_toff[j];
+                    d.active_tiles[t] = wj;
+                    d.tile_rows[t] = roff;
+                }
             }
         }
-        __syncthreads();
-        if (tid == 0) {
-            s_fresh += min(total, top);
-            s_free_top = max(top - total, 0);
-        }
-        __syncthreads();
-    }
-
-    // (5) ascending active-row and active-tile lists, new mask words
-    for (int base = 0; base < nw; base += blockDim.x) {
-        const int w = base + tid;
-        const uint32_t word = (w < nw) ? new_w[w] : 0u;
-        int nrows, ntiles;
-        const int roff = block_exclusive_scan(__popc(word), scan_scratch, &nrows);
-        const int toff = block_exclusive_scan(word != 0u, scan_scratch, &ntiles);
-        const int rb = s_rows + roff;
-        int j = 0;
-        for (uint32_t bits = word; bits; bits &= bits - 1)
-            d.active_rows[rb + j++] = (w << 5) + __ffs(bits) - 1;
-        if (word) {
-            d.active_tiles[s_tiles + toff] = w;
-            d.tile_rows[s_tiles + toff] = rb;
-        }
-        if (w < nw) d.words[w] = word;
-        __syncthreads();
-        if (tid == 0) {
-            s_rows += nrows;
-            s_tiles += ntiles;
-        }
+        need_base += tot1 >> 16;
+        rows_base += tot1 & 0xFFFF;
+        tiles_base += tot2;
         __syncthreads();
     }
     int total_over;
     block_exclusive_scan(over, scan_scratch, &total_over);
     if (tid == 0) {
-        d.counts[0] = s_rows;
-        d.counts[1] = s_tiles;
-        d.counts[2] = s_free_top;
+        d.counts[0] = rows_base;
+        d.counts[1] = tiles_base;
+        d.counts[2] = max(top2 - need_base, 0);
         d.counts[3] = total_over;
-        d.counts[4] = s_fresh;
+        d.counts[4] = min(need_base, top2);
         if (total_over) set_status(status, SF_STATUS_SLOT_OVERFLOW);
     }
 }
@@ -368,14 +387,31 @@ extern "C" int sf_mask_update(const sf_mask *masks, const sf_mask_src *srcs, int
     }
     if (n_masks == 0) return SF_OK;
     cudaStream_t st = as_stream(stream);
-    const size_t fin_smem = (size_t)2 * (max_rows / 32) * sizeof(uint32_t);
+    const size_t fin_smem = (size_t)3 * (max_rows / 32) * sizeof(uint32_t);
     if (fin_smem > 48 * 1024 &&
         cudaFuncSetAttribute(mask_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)fin_smem) != cudaSuccess)
         return SF_ERR_CUDA;
 
+    const int sms = sm_count();
     for (int first = 0; first < n_masks; first += kMaxMasksPerLaunch) {
         const int cnt = n_masks - first < kMaxMasksPerLaunch ? n_masks - first : kMaxMasksPerLaunch;
+        // Token segment length of the column-absmax pass: 512 tokens, shortened (down to 32) when
+        // the launch would otherwise give each SM fewer than ~8 CTAs, so that enough loads are in
+        // flight to cover HBM latency (a lone projection has only R / 2048 column blocks).
+        int seg_tokens = kTokensPerSeg;
+        {
+            long base = 0;
+            for (int j = 0; j < cnt; ++j) {
+                const sf_mask_src &s = srcs[first + j];
+                if (s.kind == SF_SRC_OUTPUT_BF16)
+                    base += (long)((masks[first + j].R + kColsPerCta - 1) / kColsPerCta) *
+                            ((s.n + kTokensPerSeg - 1) / kTokensPerSeg);
+            }
+            const long target = 8L * (sms > 0 ? sms : 148);
+            while (base > 0 && seg_tokens > kMinTokensPerSeg && base * (kTokensPerSeg / seg_tokens) < target)
+                seg_tokens >>= 1;
+        }
         MaskBatch batch;
         batch.n = cnt;
         int ctas = 0;
@@ -401,7 +437,7 @@ extern "C" int sf_mask_update(const sf_mask *masks, const sf_mask_src *srcs, int
             d.counts = m.counts;
             d.cta_begin = ctas;
             d.col_blocks = (m.R + kColsPerCta - 1) / kColsPerCta;
-            d.tok_segs = (s.n + kTokensPerSeg - 1) / kTokensPerSeg;
+            d.tok_segs = (s.n + seg_tokens - 1) / seg_tokens;
             if (s.kind == SF_SRC_TOKENS)
                 ctas += (s.n + kTokensPerTokCta - 1) / kTokensPerTokCta;
             else if (s.kind == SF_SRC_OUTPUT_BF16)
