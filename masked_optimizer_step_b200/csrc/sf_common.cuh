@@ -17,6 +17,13 @@ namespace sf {
 // Status word and bounded waits.
 // --------------------------------------------------------------------------------------------
 
+// Programmatic dependent launch. A grid launched with programmatic stream serialization may
+// start once every CTA of the grid before it has executed launch_dependents (or exited);
+// griddep_wait blocks until that earlier grid has completed and its memory is visible. Without
+// such a predecessor both are no-ops.
+SF_DEVICE void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+SF_DEVICE void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 SF_DEVICE void set_status(uint32_t *st, uint32_t bits)
 {
     if (st) atomicOr(st, bits);

@@ -255,6 +255,12 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+    // The launches of one call write disjoint problems, so the next one may take SMs as soon as
+    // this one's CTAs drain (its CTAs cannot share an SM with these: shared memory). Every launch
+    // reads only what the gather pass and the masks left, which were complete before the first
+    // launch of the call started.
+    griddep_launch_dependents();
+
     {   // per group: mode and units; per problem: M-tiles before it inside its group
         int units = 0;
         if (tid < b.n_group) {
@@ -468,6 +474,9 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
+    // Complete only after the launch before this one has: whatever the stream runs next then
+    // sees every launch of the call finished.
+    griddep_wait();
 }
 
 // ------------------------------------ host side ------------------------------------
@@ -636,6 +645,7 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
     int n_launch = (int)((all + payload - 1) / payload);
     DwBatch *batch = rc == SF_OK ? new DwBatch : nullptr;
     int gi = 0;
+    int n_main_launches = 0;
     for (int li = 0; rc == SF_OK && gi < ng; ++li) {
         size_t left = 0;
         for (int k = gi; k < ng; ++k) left += launch_bytes(groups[k]);
@@ -701,8 +711,23 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
         if (rc != SF_OK) break;
         const int grid = (int)(max_units < sms ? max_units : sms);
         if (grid > 0) {
-            masked_dw_kernel<<<grid, kThreads, kSmemBytes, st>>>(*batch, dev_status);
-            if (launch_status() != SF_OK) { rc = SF_ERR_CUDA; break; }
+            // launches after the first of the call overlap their predecessor's last wave
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr.val.programmaticStreamSerializationAllowed = 1;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(grid);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = kSmemBytes;
+            cfg.stream = st;
+            cfg.attrs = &attr;
+            cfg.numAttrs = n_main_launches > 0 ? 1 : 0;
+            if (cudaLaunchKernelEx(&cfg, masked_dw_kernel, *batch, dev_status) != cudaSuccess ||
+                launch_status() != SF_OK) {
+                rc = SF_ERR_CUDA;
+                break;
+            }
+            ++n_main_launches;
         }
         gi = g_end;
     }

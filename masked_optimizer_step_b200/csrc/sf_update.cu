@@ -168,6 +168,8 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
     __shared__ int s_prefix[kMaxMatsPerLaunch + 1];
     __shared__ int scan_scratch[33];
     __shared__ uint32_t max_scratch[33];
+    __shared__ int s_meta[5];
+    __shared__ float s_metaf[3];
 
     const int tid = threadIdx.x;
     for (int base = 0; base < b.n; base += kThreads) {   // prefix of active-row counts
@@ -184,30 +186,79 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
     const int total = s_prefix[b.n];
     float nan_sum = 0.0f, big = 0.0f;
 
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    // Per-row metadata is a chain of dependent loads (row id -> slot -> step count -> bias
+    // corrections). Thread 0 walks the chain of the CTA's next row one link per phase of the
+    // current row, so its latency hides behind the current row's traffic, and publishes the
+    // result in shared memory for the next iteration.
+    auto locate = [&](int item) {
         int lo = 0, hi = b.n - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (s_prefix[mid] <= item) lo = mid; else hi = mid - 1;
         }
-        const UpdDesc &d = b.d[lo];
-        const int r = d.active_rows[item - s_prefix[lo]];
-        const int slot = d.row_slot[r];
-        if (slot < 0) continue;                       // no moments for this row (overflow)
-        const int pslot = d.prow_slot ? d.prow_slot[r] : -1;
-        const int t_old = d.slot_step[slot];
+        return lo;
+    };
+    int n_lo = 0, n_r = 0, n_slot = -1, n_pslot = -1, n_t = 0;
+    float n_sc = 0.0f;
+    auto publish = [&]() {
+        const int ti = n_t + 1 < b.t_max ? n_t + 1 : b.t_max;
+        s_meta[0] = n_lo;
+        s_meta[1] = n_r;
+        s_meta[2] = n_slot;
+        s_meta[3] = n_pslot;
+        s_meta[4] = n_t;
+        s_metaf[0] = n_sc;
+        s_metaf[1] = b.bc1[ti];
+        s_metaf[2] = b.bc2[ti];
+    };
+    auto link_slot = [&]() {                        // needs n_r
+        const UpdDesc &dn = b.d[n_lo];
+        n_slot = dn.row_slot[n_r];
+        n_pslot = dn.prow_slot ? dn.prow_slot[n_r] : -1;
+        n_sc = dn.s[n_r];
+    };
+    auto link_step = [&]() {                        // needs n_slot
+        n_t = n_slot >= 0 ? b.d[n_lo].slot_step[n_slot] : 0;
+    };
+    if (tid == 0 && (int)blockIdx.x < total) {
+        n_lo = locate(blockIdx.x);
+        n_r = b.d[n_lo].active_rows[blockIdx.x - s_prefix[n_lo]];
+        link_slot();
+        link_step();
+        publish();
+    }
+
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        __syncthreads();                 // this row's metadata is published; the shared row is free
+        const UpdDesc &d = b.d[s_meta[0]];
+        const int r = s_meta[1], slot = s_meta[2], pslot = s_meta[3], t_old = s_meta[4];
+        const float sc = s_metaf[0], bc1 = s_metaf[1], bc2 = s_metaf[2];
+        const int nxt = item + gridDim.x;
+        const bool chain = tid == 0 && nxt < total;
+        if (chain) {                                 // link 1: the next row's id
+            n_lo = locate(nxt);
+            n_r = b.d[n_lo].active_rows[nxt - s_prefix[n_lo]];
+        }
+        if (slot < 0) {                              // no moments for this row (overflow)
+            if (chain) {
+                link_slot();
+                link_step();
+            }
+            __syncthreads();                         // every thread has read this row's metadata
+            if (chain) publish();
+            continue;
+        }
         const int t = t_old + 1;
-        const int ti = t < b.t_max ? t : b.t_max;
         AdamRow a;
-        a.sc = d.s[r];
+        a.sc = sc;
         a.c_self = d.c_self;
         a.c_partner = d.c_partner;
         a.beta1 = b.beta1;
         a.beta2 = b.beta2;
         a.omb1 = b.omb1;
         a.omb2 = b.omb2;
-        a.bc1 = b.bc1[ti];
-        a.bc2 = b.bc2[ti];
+        a.bc1 = bc1;
+        a.bc2 = bc2;
         a.eps = b.eps;
         a.nlr = -b.lr;
         a.nlrwd = __fmul_rn(-b.lr, b.wd);
@@ -244,6 +295,7 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
                 wrow4[2 * j + 1] = make_float4(wn[4], wn[5], wn[6], wn[7]);
             }
         }
+        if (chain) link_slot();                      // link 2: the next row's slot and scale
 
         // new per-row scale from the row absmax (non-negative floats order as unsigned ints);
         // the reduction's barriers also publish the shared-memory row to every thread
@@ -251,6 +303,7 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         const float sp = __fdiv_rn(rmax, 127.0f);
         const float rcp = __frcp_rn(sp);
         const bool fast = sp != 0.0f && isfinite(rcp);
+        if (chain) link_step();                      // link 3: the next row's step count
 
         // ---- pass 2: requantise from shared memory, write q, delta and the live row ----
         int8_t *qout = d.q + (size_t)r * C;
@@ -289,7 +342,7 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
             d.s[r] = sp;
             d.slot_step[slot] = t;
         }
-        __syncthreads();                 // the shared row is reused by the next item
+        if (chain) publish();                        // link 4: bias corrections; ready for the next row
     }
     if (nan_sum != 0.0f || !(big < 65520.0f)) set_status(status, SF_STATUS_NONFINITE);
 }
