@@ -53,6 +53,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps (capped at 20)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--chunks", type=int, default=1,
+                    help="layer chunks per step: chunk c's masks run on a side stream while earlier "
+                         "chunks' dW and update run on the main stream (1, the default and the "
+                         "fastest measured: one call per stage on one stream)")
     ap.add_argument("--sweep", action="store_true",
                     help="density sweep of one 11008 x 4096 projection (T = 4096), scattered and "
                          "clustered rows, with a dense bf16 GEMM and a fused dense Adam as context; "
@@ -89,6 +93,8 @@ def workload_config(args):
         "hidden": 4096, "ffn": 11008, "vocab": 32000,
         "l2": "no flush needed: each step reads ~14 GB of resident inputs (L2 is 126 MB)",
         "parallelism": "replicas",
+        "schedule": f"{args.chunks} layer chunks, masks on a side stream overlapping earlier chunks' dW and update"
+                    if args.chunks > 1 else "one call per stage, one stream",
     }
 
 
@@ -465,7 +471,7 @@ def main():
     torch.cuda.set_device(local)
     device = f"cuda:{local}"
     from masked_optimizer_step_b200 import binding as sf
-    from masked_optimizer_step_b200.model import SparseModel, StepPlan
+    from masked_optimizer_step_b200.model import Pipeline, SparseModel
     sf.load()
 
     T = args.tokens
@@ -480,11 +486,10 @@ def main():
         b["tokens"] = tok_dev[prior]
     ws = torch.zeros(sf.sf_embed_grad_ws_bytes(T, model.emb.mask.slot_cap) // 4 + 64, dtype=torch.int32,
                      device=device)
-    plans = [StepPlan(model, b, ws) for b in banks]
+    plans = [Pipeline(model, b, ws, chunks=args.chunks) for b in banks]
     hp = sf.AdamParams(device=device)
     status = sf.status_word(device)
     stream = torch.cuda.current_stream()
-    sp = stream.cuda_stream
     st_ptr = status.data_ptr()
 
     # the conductor sees 20 prior windows before the first step
@@ -492,30 +497,17 @@ def main():
     for w in range(prior):
         sf.sf_mask_update([model.emb.mask], [emb_src[w]], 0.01, status)
 
-    def step(k, events=None):
-        plan = plans[k % 2]
-        plan.set_tokens(tok_dev[prior + k])
-        plan.set_coupling(36.0 * k)
-        if events is not None:
-            events[0].record(stream)
-        plan.masks(st_ptr, sp)
-        if events is not None:
-            events[1].record(stream)
-        plan.dw(st_ptr, sp)
-        if events is not None:
-            events[2].record(stream)
-        plan.embed(st_ptr, sp)
-        if events is not None:
-            events[3].record(stream)
-        plan.update(hp, st_ptr, sp)
-        if events is not None:
-            events[4].record(stream)
+    def step(k, timing=None):
+        pipe = plans[k % 2]
+        pipe.set_tokens(tok_dev[prior + k])
+        pipe.set_coupling(36.0 * k)
+        pipe.step(hp, st_ptr, stream, timing)
 
     for k in range(args.warmup):
         step(k)
     torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    timing = []
     counts_log = torch.zeros((args.steps,) + tuple(model.counts.shape), dtype=torch.int32, device=device)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -527,7 +519,7 @@ def main():
     time.sleep(0.1)
     t_start.record(stream)
     for k in range(args.steps):
-        step(args.warmup + k, ev[k])
+        step(args.warmup + k, timing)
         counts_log[k].copy_(model.counts, non_blocking=True)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -535,10 +527,10 @@ def main():
     if world > 1:
         dist.barrier()
     ms_total = t_start.elapsed_time(t_end)
+    stage_names = ("masks", "masked_dw", "embed_grad", "sparse_update")
     stage_ms = np.zeros(4)
-    for k in range(args.steps):
-        for j in range(4):
-            stage_ms[j] += ev[k][j].elapsed_time(ev[k][j + 1])
+    for name, e0, e1 in timing:
+        stage_ms[stage_names.index(name)] += e0.elapsed_time(e1)
     counts = counts_log.cpu().numpy()
     work = [step_work(model, counts[k], T) for k in range(args.steps)]
     rows_updated = sum(w["rows_updated"] for w in work)
@@ -696,13 +688,10 @@ def run_e2e(args, model, banks, plans, hp, tok_dev, prior, stream, device, world
             tok_bufs[b].copy_(tok_host[prior + (base + k) % (tok_host.shape[0] - prior)], non_blocking=True)
             copied[b].record(cs)
         stream.wait_event(copied[b])
-        plan = plans[b]
-        plan.set_tokens(tok_bufs[b])
-        plan.set_coupling(36.0 * (base + k))
-        plan.masks(status.data_ptr(), sp)
-        plan.dw(status.data_ptr(), sp)
-        plan.embed(status.data_ptr(), sp)
-        plan.update(hp, status.data_ptr(), sp)
+        pipe = plans[b]
+        pipe.set_tokens(tok_bufs[b])
+        pipe.set_coupling(36.0 * (base + k))
+        pipe.step(hp, status.data_ptr(), stream)
         consumed[b].record(stream)
         result[:1].copy_(status, non_blocking=True)
         result[1:].copy_(model.counts.view(-1), non_blocking=True)

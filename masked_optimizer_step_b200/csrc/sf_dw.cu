@@ -44,7 +44,10 @@ constexpr int BM = 128;                 // rows per unit
 constexpr int BN = 256;                 // columns per unit
 constexpr int BK = 64;                  // tokens per pipeline stage
 constexpr int UMMA_K = 16;              // K of one tcgen05.mma kind::f16
-constexpr int STAGES = 4;
+#ifndef SF_DW_STAGES
+#define SF_DW_STAGES 4
+#endif
+constexpr int STAGES = SF_DW_STAGES;
 constexpr int A_TILE_BYTES = 32 * BK * 2;          // 32 rows x 64 tokens (64 B rows)
 constexpr int A_STAGE_BYTES = 4 * A_TILE_BYTES;    // 16 KB
 constexpr int B_BOX_BYTES = 64 * BK * 2;           // 64 columns x 64 tokens (128 B rows)
@@ -308,8 +311,8 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             }
             int stage = 0;
             uint32_t phase = 0;
-            bool issued[STAGES] = {false, false, false, false};
-            uint32_t issued_parity[STAGES] = {0, 0, 0, 0};
+            bool issued[STAGES] = {};
+            uint32_t issued_parity[STAGES] = {};
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
                 const Unit x = decode(u, sp, b);
