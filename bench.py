@@ -57,6 +57,10 @@ def parse():
                     help="layer chunks per step: chunk c's masks run on a side stream while earlier "
                          "chunks' dW and update run on the main stream (1, the default and the "
                          "fastest measured: one call per stage on one stream)")
+    ap.add_argument("--config", choices=["c0", "c1", "c2"], default=None,
+                    help="time one of the smaller workloads instead of the headline step (one JSON line "
+                         "each, not the headline metric): c0 the tiny projection, c1 the embedding "
+                         "path, c2 one 7B-shaped layer at 4,096 tokens (scattered and clustered)")
     ap.add_argument("--sweep", action="store_true",
                     help="density sweep of one 11008 x 4096 projection (T = 4096), scattered and "
                          "clustered rows, with a dense bf16 GEMM and a fused dense Adam as context; "
@@ -455,12 +459,135 @@ def run_sweep(args):
     return 0
 
 
+def _stage_line(model, pipe, hp, status, T, steps, warm, stream, before_step=None):
+    """Time `steps` steps of a Pipeline after `warm` warm-up steps; returns (ms per step, stage ms
+    per step, list of per-step work dicts)."""
+    import torch
+    for k in range(warm):
+        if before_step:
+            before_step(k)
+        pipe.step(hp, status.data_ptr(), stream)
+    torch.cuda.synchronize()
+    timing, counts = [], []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    log = torch.zeros((steps,) + tuple(model.counts.shape), dtype=torch.int32, device=model.device)
+    t0.record(stream)
+    for k in range(steps):
+        if before_step:
+            before_step(warm + k)
+        pipe.step(hp, status.data_ptr(), stream, timing)
+        log[k].copy_(model.counts, non_blocking=True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    names = ("masks", "masked_dw", "embed_grad", "sparse_update")
+    st = np.zeros(4)
+    for name, e0, e1 in timing:
+        st[names.index(name)] += e0.elapsed_time(e1)
+    work = [step_work(model, c, T) for c in log.cpu().numpy()]
+    return t0.elapsed_time(t1) / steps, st / steps, work
+
+
+def run_config(args):
+    """The smaller workloads: c0 the tiny projection (256 x 512, 128 tokens, fixed 3%-row mask,
+    3 Adam steps), c1 the embedding path (32,000 x 4,096 table, 8 x 512 Zipf(1.1) tokens, seed 1,
+    20 prior conductor windows; conductor, row gradient and update), c2 one 7B-shaped layer
+    (4,096 tokens, tracker masks at ~1% scattered and clustered, coupled pairs)."""
+    import torch
+    from masked_optimizer_step_b200 import binding as sf
+    from masked_optimizer_step_b200 import synth
+    from masked_optimizer_step_b200.model import INPUT_OF, Pipeline, SparseModel
+    sf.load()
+    device = "cuda:0"
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    hp = sf.AdamParams(device=device)
+    status = sf.status_word(device)
+    steps, warm = max(args.steps, 3), max(args.warmup, 3)
+
+    def emit(name, workload, T, model, ms, st, work):
+        rows = sum(w["rows_updated"] for w in work) / len(work)
+        upd = sum(w["update_bytes"] for w in work) / len(work)
+        line = {"config": name, "workload": workload, "ms_per_step": ms,
+                "active_row_updates_per_s": rows / (ms / 1e3), "rows_updated_per_step": rows,
+                "ms": dict(zip(("masks", "masked_dw", "embed_grad", "sparse_update"), map(float, st))),
+                "update_gbs": upd / (st[3] / 1e3) / 1e9 if st[3] > 0 else None,
+                "update_frac_hbm": upd / (st[3] / 1e3) / 1e9 / hbm if st[3] > 0 else None,
+                "device_status": int(status.cpu()[0])}
+        dwb = sum(w["dw_bytes"] for w in work) / len(work)
+        if st[1] > 0:
+            line["masked_dw_tflops_useful"] = sum(w["dw_flops_useful"] for w in work) / len(work) / (st[1] / 1e3) / 1e12
+            line["masked_dw_gbs"] = dwb / (st[1] / 1e3) / 1e9
+        if st[0] > 0 and model.projs:
+            line["tracker_gbs"] = sum(w["tracker_bytes"] for w in work) / len(work) / (st[0] / 1e3) / 1e9
+        print(json.dumps(line), flush=True)
+
+    if args.config == "c0":
+        shapes = (("down", 256, 512),)           # an unpaired projection
+        model = SparseModel(1, vocab=0, layer_shapes=shapes, slot_frac=0.25, device=device)
+        W = torch.from_numpy(synth.weights_f32(synth.rng(0, "weights"), 256, 512)).to(device)
+        mat = model.projs[0].mat
+        sf.sf_quantize_init(W, mat)
+        sf.sf_mask_init(mat.mask)
+        T = 128
+        words = torch.from_numpy(synth.tiny_projection_mask(0, 256).view(np.int32)).to(device)
+        dX = torch.from_numpy(synth.normal_bf16(synth.rng(0, "dx", 0), (T, 256)).view(np.int16)).view(torch.bfloat16).to(device)
+        A = torch.from_numpy(synth.normal_bf16(synth.rng(0, "act", 0), (T, 512)).view(np.int16)).view(torch.bfloat16).to(device)
+        inputs = {"tokens": None, "dY": None, "Y": [dX], "dX": [dX], "A": [A]}
+        pipe = Pipeline(model, inputs, None)
+        pipe.plans[0].src_arr[0] = sf.sf_mask_src(sf.SF_SRC_WORDS, 0, 0, words.data_ptr())
+        ms, st, work = _stage_line(model, pipe, hp, status, T, steps, warm, stream)
+        emit("C0", "tiny projection: W 256x512, 128 tokens, fixed 3%-row mask (one full and five empty "
+                   "tiles), seed 0", T, model, ms, st, work)
+        return 0
+    if args.config == "c1":
+        model = SparseModel(0, vocab=32000, emb_slots=4096, device=device)
+        model.init(1)
+        T = 8 * 512
+        g = synth.rng(1, "tokens")
+        toks = torch.from_numpy(np.stack([synth.zipf_ids(g, T, 32000) for _ in range(20 + warm + steps)])).to(device)
+        for w in range(20):
+            sf.sf_mask_update([model.emb.mask], [sf.make_src(sf.SF_SRC_TOKENS, toks[w], n=T)], 0.01, status)
+        dY = synth.device_normal_bf16((T, 4096), 1, "dy", device=device)
+        ws = torch.zeros(sf.sf_embed_grad_ws_bytes(T, model.emb.mask.slot_cap) // 4 + 64, dtype=torch.int32,
+                         device=device)
+        inputs = {"tokens": toks[20], "dY": dY, "Y": [], "dX": [], "A": []}
+        pipe = Pipeline(model, inputs, ws)
+        ms, st, work = _stage_line(model, pipe, hp, status, T, steps, warm, stream,
+                                   before_step=lambda k: pipe.set_tokens(toks[20 + k]))
+        emit("C1", "embedding path: 32000x4096 int8+residual table, 8x512 Zipf(1.1) tokens per step, "
+                   "20 prior conductor windows, seed 1", T, model, ms, st, work)
+        return 0
+    # c2: one 7B-shaped layer at 4,096 tokens
+    T = 4096
+    for kind in ("scattered", "clustered"):
+        model = SparseModel(1, vocab=0, device=device)
+        model.init(2)
+        projs = [(p.layer, p.name, p.mat.R, p.mat.C, INPUT_OF[p.name]) for p in model.projs]
+        bank = synth.step_bank(projs, T, kind, 0, 2, device=device)
+        pipe = Pipeline(model, bank, None)
+        ms, st, work = _stage_line(model, pipe, hp, status, T, steps, warm, stream,
+                                   before_step=lambda k: pipe.set_coupling(36.0 * k))
+        emit("C2", f"one 7B-shaped layer (q,k,v,o 4096x4096; gate,up 11008x4096; down 4096x11008), 4096 "
+                   f"tokens, ~1% {kind} tracker masks, coupled pairs, seed 2", T, model, ms, st, work)
+        del model, bank, pipe
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.config:
+        return run_config(args)
     rank, world, local = dist_env()
     import torch
     import torch.distributed as dist

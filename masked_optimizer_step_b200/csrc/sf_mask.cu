@@ -141,14 +141,14 @@ mask_accum_kernel(const __grid_constant__ MaskBatch b, uint32_t *status)
 
 // Finalize, one CTA per mask. Phase 2 runs one warp per 32-row tile (lane = row) and issues the
 // loads of kBatch tiles before using any of them, so a warp has several independent DRAM round
-// trips in flight; the new, released and needing-a-slot bit masks of every tile stay in shared
+// trips in flight (32 registers: two CTAs per SM, so 296 masks finalize in one wave); the new, released and needing-a-slot bit masks of every tile stay in shared
 // memory. The slot sweeps and the lists then go over rounds of kRound words: a block scan of the
 // per-word counts gives every tile its offsets, and a warp per tile writes its rows' entries,
 // touching global memory only for rows that change state.
-constexpr int kBatch = 8;
+constexpr int kBatch = 4;
 constexpr int kRound = 512;       // words per scan round; per-round sums stay below 2^15 per field
 
-__global__ void __launch_bounds__(kFinalizeThreads)
+__global__ void __launch_bounds__(kFinalizeThreads, 2)   // two per SM: a call's masks fit one wave
 mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *status)
 {
     extern __shared__ uint32_t smem_words[];
