@@ -720,8 +720,16 @@ def main():
     kernels = {"masks": "sf_mask_update: mask_accum_kernel + mask_finalize_kernel",
                "masked_dw": "sf_masked_dw: dw_gather_kernel + 3 x masked_dw_kernel",
                "sparse_update": "sf_sparse_update: update_kernel"}
+    traffic_rate = traffic / (d["ms_per_step"] / 1e3) / 1e9 if traffic else None
     roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
                 "frac": d["frac"], "traffic": traffic, "traffic_unit": "bytes per step (one call)",
+                "traffic_gbs": traffic_rate,
+                "traffic_frac": traffic_rate / hbm if traffic_rate else None,
+                "traffic_note": "DRAM bytes the call actually moves (ncu) over its event-timed duration: the "
+                                "row gather reads dX at DRAM granularity (~128 B per 64-column window "
+                                "holding an active row), so traffic exceeds the 2 B per gathered element "
+                                "counted in the algorithmic bytes" if d["bound"] == "hbm" and dominant == "masked_dw"
+                                else None,
                 "kernel": kernels[dominant], "peak_source": peak_src,
                 "peak_kind": "sustained bf16 (kernel timed inside a long step)" if d["bound"] == "tensor" else "hbm copy",
                 "algorithmic": d["algorithmic"]}
