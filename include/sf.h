@@ -258,10 +258,9 @@ int sf_adam_tables(float beta1, float beta2, int t_max, float *bc1, float *bc2,
 int sf_sparse_update(const sf_matrix *mats /* host [n_mats] */, int n_mats,
                      const sf_adam *hp /* host */, uint32_t *dev_status, sf_stream stream);
 
-/* ---- sf_checkpoint_save / sf_checkpoint_restore: section 2.6, "Checkpoint and rewind" -----
- * The optimizer keeps a checkpoint of the active rows only, so a checkpoint costs no more than
- * the active set, and restores it when the loss rebounds (the policy that decides when is host
- * logic). A checkpoint of one matrix is a snapshot, at save time, of each active row (ascending):
+/* ---- sf_checkpoint_save / sf_checkpoint_restore: section 2.6 --------------------------------
+ * Only rows in the active set are saved, so a snapshot is as small as that set, and it is put
+ * back when the loss rebounds (the policy that decides when is host logic). A checkpoint of one matrix is a snapshot, at save time, of each active row (ascending):
  *   rows[k] the row, q[k*C..] int8, s[k], delta[k*C..] fp32, m, v[k*C..] fp16 bits (zeros for a
  *   row without a slot), step[k] its Adam step count; *count the rows saved (device).
  * Buffers hold `cap` rows; a save with more active rows keeps the first cap and sets

@@ -1,7 +1,7 @@
 // sf_ckpt.cu -- checkpoint and rewind of the active rows.
 //
-// "Sparse-First Fine-Tuning" (tensorwirelabs.com), section 2.6 (Checkpoint and rewind): the
-// optimizer checkpoints only the active rows, so a checkpoint costs no more than the active set;
+// "Sparse-First Fine-Tuning" (tensorwirelabs.com), section 2.6: only rows in the active set are
+// saved, so a snapshot is as small as that set;
 // when the loss rebounds past a threshold the checkpoint is restored. A checkpoint here is a
 // snapshot, at save time, of every active row's q, s, delta, moments and Adam step count, in
 // ascending row order. Restoring writes q, s and delta back, rebuilds the row's bf16 live

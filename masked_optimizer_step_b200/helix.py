@@ -1,16 +1,16 @@
 """Host-side decisions of a sparse-first step: the rewind policy and the Helix coupling schedule.
 
 "Sparse-First Fine-Tuning" (tensorwirelabs.com):
-  * section 2.6 (Checkpoint and rewind): when to save the active-row checkpoint, when a new loss
-    minimum opens a watch, and when the watch ends in a rewind (restore, stride back to 1, skip
-    the step) or in accepting the minimum;
+  * section 2.6: when to save the active-row snapshot, when a fresh low of the loss starts a
+    watch, and whether that watch closes with a rewind (restore, stride back to 1, skip the step)
+    or by keeping the low;
   * sections 2.4 / 2.5 (The coupled update; Adapting to the loss trend): the rotating phase, the
     Fibonacci stride driven by the loss trend, the two channel weights and their slow modulation,
-    the non-periodic phase from a point walking an elliptic curve, and the weight decay scaled by
+    the non-periodic phase read off a point that steps along an elliptic curve, and the weight decay scaled by
     the cosine of the pitch angle.
 
 Everything here is host arithmetic on scalars that the previous step left behind (its loss); it
-reads nothing from the device in the middle of a step (section 2.6, last paragraph). The
+reads nothing back from the device while a step is running (section 2.6, last paragraph). The
 formula that turns phase, exposure and channel weights into the effective gradients is not in
 the text the pages give (it is an image that did not survive extraction), so `Helix.coefficients`
 is a reading: the kernel takes any per-pair linear mix, and this is one that follows every
@@ -31,8 +31,8 @@ TURN_MOD = 0.10                      # modulation of the channel weights at the 
 TEN_TURN_MOD = 0.05                  # ... and at the scale of ten turns
 STRENGTH = {"gate-up": 0.6, "q-o": 0.4, "k-v": 0.4}
 
-CKPT_GATE = 0.10                     # save while the loss is within 10% of the last checkpoint
-WATCH_STEPS = 10                     # a new minimum opens a ten-step watch
+CKPT_GATE = 0.10                     # save while the loss stays inside +-10% of the saved loss
+WATCH_STEPS = 10                     # length of the watch that a fresh loss low starts
 REBOUND = 0.15                       # rewind when the loss ends the watch >15% above the minimum
 MAX_RECOVERIES = 3                   # rewinds allowed per minimum
 
@@ -52,7 +52,7 @@ def fibonacci_rungs(cap: int = FIB_CAP) -> list[int]:
 @dataclass
 class Action:
     """What the host does before launching the next step."""
-    save: bool = False               # take a checkpoint of the active rows now
+    save: bool = False               # snapshot the active rows now
     restore: bool = False            # restore the checkpoint (then reset the stride)
     skip: bool = False               # skip this step's update
     event: str = ""                  # "", "save", "watch", "rewind", "accept", "exhausted"
@@ -70,9 +70,9 @@ class RewindPolicy:
         further losses, resets the count of recoveries and is saved if the gate allows.
       * Inside a watch only new minima are saved, so that a rewind goes back to the minimum's
         state and not to a state from the rise that the watch is judging.
-      * At the end of the watch, a loss above (1 + REBOUND) x the minimum rewinds: restore, stride
+      * When the watch runs out, a loss above (1 + REBOUND) x the minimum rewinds: restore, stride
         back to 1, skip the step, count one recovery and watch again for the same minimum.
-      * Otherwise the minimum is accepted: the watch closes and the minimum's loss becomes the
+      * If not, the low stands: the watch closes and the minimum's loss becomes the
         checkpoint's reference loss, so the gate measures later losses from it. After
         MAX_RECOVERIES rewinds the current state is accepted as it is: it is saved and becomes the
         reference minimum.
@@ -101,7 +101,7 @@ class RewindPolicy:
     def _decide(self, loss: float) -> Action:
         if not math.isfinite(loss):
             return Action(restore=True, skip=True, event="rewind") if self.ckpt_loss is not None else Action()
-        if loss < self.best:                                 # a new minimum opens a watch
+        if loss < self.best:                                 # a fresh low starts a watch
             self.best = loss
             self.watch_left = self.watch_steps
             self.recoveries = 0
@@ -113,7 +113,7 @@ class RewindPolicy:
             self.watch_left -= 1
             if self.watch_left > 0:
                 return Action()
-            if loss > (1.0 + self.rebound) * self.best:      # end of the watch: rebound
+            if loss > (1.0 + self.rebound) * self.best:      # watch over: the loss rebounded
                 if self.recoveries < self.max_recoveries:
                     self.recoveries += 1
                     self.watch_left = self.watch_steps
@@ -194,7 +194,7 @@ class Stride:
 
 
 # ---------------------------------------------------------------------------------------------
-# section 2.4: the slow non-periodic phase psi (a point walking an elliptic curve)
+# section 2.4: the slow non-periodic phase psi (a point stepping along an elliptic curve)
 # ---------------------------------------------------------------------------------------------
 
 @dataclass

@@ -405,7 +405,7 @@ void orc_rebuild_rows(int R, int C, const int8_t *q, const float *s, const float
 /* ------------------------------------------------------------------------------------------ */
 
 /*
- * Section 2.6 keeps a checkpoint of the active rows only. Reading taken: a checkpoint is a
+ * Section 2.6 saves rows of the active set only. Reading taken: a checkpoint is a
  * snapshot, at save time, of every active row's storage and optimizer state: its row id, q, s,
  * delta, m, v and step count. Rows are saved in ascending row order. Returns the rows saved.
  * Buffers hold cap rows (rows beyond cap are not saved; the return value says how many were).

@@ -204,7 +204,7 @@ def test_steady_descent_saves_every_minimum():
     assert not any(a.restore for a in acts)
 
 
-def test_rebound_past_15_percent_rewinds_at_the_end_of_the_watch():
+def test_rebound_past_15_percent_rewinds_when_the_watch_runs_out():
     p = hx.RewindPolicy()
     acts = _events(p, [1.0, 0.95] + [1.0] * 9 + [1.1])        # 1.1 > 1.15 * 0.95 = 1.0925
     assert acts[1].save and acts[1].event == "watch"
