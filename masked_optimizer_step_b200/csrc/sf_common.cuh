@@ -160,6 +160,9 @@ SF_DEVICE bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
     }
 }
 
+// Ask L2 to fetch the line holding p (no register result; the load that follows hits L2).
+SF_DEVICE void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 SF_DEVICE void prefetch_tmap(const CUtensorMap *m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

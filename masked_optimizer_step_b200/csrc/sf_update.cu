@@ -276,6 +276,23 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         // ---- pass 1: rebuild, mix, Adam; moments out, new weight to shared memory ----
         float amax = 0.0f;
         for (int j0 = tid; j0 < nchunks; j0 += kThreads * UNROLL) {
+            {   // the thread's next chunk: into L2 now, so its loads next iteration hit L2. One lane in
+                // each group that shares a 128-byte line asks for it.
+                const int jn = j0 + kThreads * UNROLL;
+                if (jn < nchunks) {
+                    const int cn = jn << 3;
+                    if ((tid & 3) == 0) {
+                        prefetch_l2(drow + cn);
+                        prefetch_l2(grow + cn);
+                        if (partner) prefetch_l2(prow + cn);
+                    }
+                    if ((tid & 7) == 0 && moments) {
+                        prefetch_l2(mrow + cn);
+                        prefetch_l2(vrow + cn);
+                    }
+                    if ((tid & 15) == 0) prefetch_l2(qrow + cn);
+                }
+            }
             Chunk k[UNROLL];
 #pragma unroll
             for (int u = 0; u < UNROLL; ++u) {
