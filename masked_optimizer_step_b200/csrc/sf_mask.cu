@@ -26,6 +26,10 @@ constexpr int kColsPerThread = 8;                            // one 16-byte load
 constexpr int kColsPerCta = kAccumThreads * kColsPerThread;  // 2048
 constexpr int kTokensPerSeg = 512;
 constexpr int kMinTokensPerSeg = 32;
+#ifndef SF_MASK_PREFETCH_ROWS
+#define SF_MASK_PREFETCH_ROWS 8
+#endif
+constexpr int kPrefetchRows = SF_MASK_PREFETCH_ROWS;   // prefetch distance of the column-max pass
 constexpr int kTokensPerTokCta = kAccumThreads * 8;          // histogram: 8 ids per thread
 constexpr int kFinalizeThreads = 1024;
 constexpr int kMaxRows = 262144;                             // three bit masks per tile fit in smem
@@ -105,6 +109,12 @@ mask_accum_kernel(const __grid_constant__ MaskBatch b, uint32_t *status)
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
     int t = t0;
     for (; t + 8 <= t1; t += 8) {
+        // token rows kPrefetchRows ahead of this batch, into L2 (one lane per 128-byte line): the
+        // loads in flight per SM are register-limited, the prefetches are not
+        if ((threadIdx.x & 7) == 0 && t + kPrefetchRows + 8 <= t1) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) prefetch_l2(Y + (size_t)(t + kPrefetchRows + j) * d.ld + c0);
+        }
         uint4 v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
