@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: same as --steps (capped at 20)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense GEMM + dense Adam context line")
     ap.add_argument("--chunks", type=int, default=1,
                     help="layer chunks per step: chunk c's masks run on a side stream while earlier "
                          "chunks' dW and update run on the main stream (1, the default and the "
@@ -66,6 +67,16 @@ def parse():
                          "clustered rows, with a dense bf16 GEMM and a fused dense Adam as context; "
                          "prints one JSON line per point (not the headline metric)")
     return ap.parse_args()
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def dist_env():
@@ -238,15 +249,19 @@ def step_work(model, counts, T):
 # CPU oracle on a bounded sample (rank 0 only)
 # ---------------------------------------------------------------------------------------------
 
-def oracle_sample(model, bank, T, tokens, kind, max_rows=None, with_embed=True, projs=("q", "o")):
-    """Run the oracle, as it stands, on layer 0's `projs` and the embedding stage; returns
+def oracle_sample(model, bank, T, tokens, kind, max_rows=None, with_embed=True,
+                  projs=("q", "k", "v", "o", "gate", "up", "down")):
+    """Run the oracle, as it stands, on layer 0's `projs` (row trackers, masked dW, then the
+    coupled update of the pairs at the first step's mix) and the embedding stage; returns
     (seconds, active-row updates)."""
     import torch
     import oracle as orc
     from masked_optimizer_step_b200 import synth
+    from masked_optimizer_step_b200.model import PARTNER, STRENGTH
     hp = orc.AdamHP()
     rows_done = 0
     t_total = 0.0
+    states, grads = {}, {}
     for name in projs:
         i = model.index[(0, name)]
         m = model.projs[i].mat
@@ -263,10 +278,19 @@ def oracle_sample(model, bank, T, tokens, kind, max_rows=None, with_embed=True, 
             rows = rows[:max_rows]
             words = synth.words_from_rows(m.R, rows)
         st.set_mask(words)
-        g = orc.masked_dw(dX, A, words, np.zeros((m.R, m.C))).astype(np.float32)
-        orc.update(st, g, hp)
+        grads[name] = orc.masked_dw(dX, A, words, np.zeros((m.R, m.C))).astype(np.float32)
         t_total += time.perf_counter() - t0
+        states[name] = st
         rows_done += len(rows)
+    for name in projs:
+        other = PARTNER.get(name)
+        t0 = time.perf_counter()
+        if other in states:
+            orc.update(states[name], grads[name], hp, partner=states[other], pg=grads[other],
+                       c_self=1.0, c_partner=float(np.float32(STRENGTH[name])))
+        else:
+            orc.update(states[name], grads[name], hp)
+        t_total += time.perf_counter() - t0
     if with_embed and model.emb is not None:
         dY = bank["dY"].cpu().view(torch.int16).numpy().view(np.uint16)
         V, H = model.emb.R, model.emb.C
@@ -325,7 +349,8 @@ def run_reference(args):
             t_total += dt
             rows_total += len(act)
     value = rows_total / t_total
-    cpu = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+    cpu = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "cpu_model": cpu_model(),
+           "host_cores": os.cpu_count(),
            "sample": f"per step: layer-0 q projection (4096x4096, {T} tokens): row tracker over all "
                      f"outputs, then masked dW and fused update of 8 of its active rows"}
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
@@ -457,6 +482,56 @@ def run_sweep(args):
              "peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": tf_sus}}
     print(json.dumps(dense), flush=True)
     return 0
+
+
+def dense_context(layers: int, T: int, device, reps: int = 5):
+    """Dense reference step for context: the seven projections' weight gradients as cuBLAS bf16
+    GEMMs (torch.matmul) and one fused dense fp32 Adam step (torch.optim.Adam(fused=True)) over
+    one layer, plus the embedding table's dense Adam; the layer's time is multiplied by the layer
+    count (a dense fp32 Adam state for the whole model, 16 B per parameter, does not fit beside
+    the sparse model on one GPU)."""
+    import torch
+    from masked_optimizer_step_b200 import synth
+    from masked_optimizer_step_b200.model import LLAMA_7B_LAYER
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ins = {C: synth.device_normal_bf16((T, C), SEED, "act", 9, C, device=device) for C in (4096, 11008)}
+    outs = [(synth.device_normal_bf16((T, R), SEED, "dx", 9, i, device=device), ins[C])
+            for i, (_, R, C) in enumerate(LLAMA_7B_LAYER)]
+    gemm_ms = timed(lambda: [torch.matmul(dx.t(), a) for dx, a in outs])
+    flops = sum(2.0 * T * R * C for _, R, C in LLAMA_7B_LAYER)
+    del outs, ins
+    params = [torch.nn.Parameter(torch.zeros((R, C), device=device)) for _, R, C in LLAMA_7B_LAYER]
+    for q in params:
+        q.grad = torch.zeros_like(q)
+    opt = torch.optim.Adam(params, lr=1e-4, fused=True)
+    adam_ms = timed(opt.step)
+    n_layer = sum(R * C for _, R, C in LLAMA_7B_LAYER)
+    del opt, params
+    emb = torch.nn.Parameter(torch.zeros((32000, 4096), device=device))
+    emb.grad = torch.zeros_like(emb)
+    opt = torch.optim.Adam([emb], lr=1e-4, fused=True)
+    emb_ms = timed(opt.step)
+    del opt, emb
+    torch.cuda.empty_cache()
+    return {"ms_per_step_extrapolated": layers * (gemm_ms + adam_ms) + emb_ms,
+            "per_layer": {"dw_gemm_ms": gemm_ms, "dw_gemm_tflops": flops / (gemm_ms / 1e3) / 1e12,
+                          "adam_ms": adam_ms, "adam_gbs": n_layer * 28 / (adam_ms / 1e3) / 1e9},
+            "embedding_adam_ms": emb_ms,
+            "note": "one layer timed (7 bf16 GEMMs dX^T A at the step's token count + fused fp32 Adam, "
+                    "28 B/param), times the layer count, plus the embedding's Adam; context, not a baseline"}
 
 
 def _stage_line(model, pipe, hp, status, T, steps, warm, stream, before_step=None):
@@ -748,6 +823,8 @@ def main():
         "device_status": dev_status,
     }
 
+    if not args.no_dense and rank == 0:
+        out["dense_context"] = dense_context(args.layers, T, device)
     # ---- e2e: inputs from pinned host buffers every step, result read back every step ----
     if not args.no_e2e:
         out["e2e"] = run_e2e(args, model, banks, plans, hp, tok_dev, prior, stream, device, world, dist)
@@ -757,7 +834,8 @@ def main():
         orc.build()
         secs, rows = oracle_sample(model, banks[0], T, toks[: prior + 1], args.masks)
         out["cpu_baseline"] = {"value": rows / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
-                               "sample": "layer-0 q and o projections (row tracker, masked dW, fused "
+                               "cpu_model": cpu_model(), "host_cores": os.cpu_count(),
+                               "sample": "layer 0, all seven projections (row trackers, masked dW, coupled "
                                          "update of all their active rows) and the embedding stage "
                                          "(conductor over 21 windows, row gradient, update), one step",
                                "seconds": secs, "rows": rows}
