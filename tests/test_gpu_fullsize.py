@@ -1,7 +1,8 @@
 """Parity at the full 7B shape, in the launch configuration bench.py times.
 
-One step of the 32-layer model (plus the 32,000-row embedding, 2,048 tokens, scattered ~1%
-masks) runs through the same StepPlan calls as the benchmark: 225 masks in one call, the masked
+One step of the 32-layer model (plus the 32,000-row embedding, 2,048 tokens, ~1% masks, once
+scattered and once clustered into whole tiles) runs through the same StepPlan calls as the
+benchmark: 225 masks in one call, the masked
 dW of all 224 projections in one call, the embedding-row gradient, and one grouped update. The
 oracle then recomputes sampled outputs one by one:
   - conductor charges, masks and lists over 21 windows (all 32,000 rows), and the trackers of
@@ -34,13 +35,15 @@ def _bits(t):
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-@pytest.fixture(scope="module")
-def step_state():
+@pytest.fixture(scope="module", params=["scattered", "clustered"])
+def step_state(request):
+    """Scattered rows put every dW group in row mode; clustered whole tiles put them in tile mode."""
     torch.cuda.set_device(0)
+    torch.cuda.empty_cache()
     model = SparseModel(32, device=DEV)
     model.init(SEED)
     projs = [(p.layer, p.name, p.mat.R, p.mat.C, INPUT_OF[p.name]) for p in model.projs]
-    bank = synth.step_bank(projs, T, "scattered", 0, SEED, device=DEV)
+    bank = synth.step_bank(projs, T, request.param, 0, SEED, device=DEV)
     toks = synth.token_stream(SEED, PRIOR + 1, T)
     tok_dev = torch.from_numpy(toks).to(DEV)
     srcs = [sf.make_src(sf.SF_SRC_TOKENS, tok_dev[w], n=T) for w in range(PRIOR)]
