@@ -42,8 +42,12 @@ namespace {
 
 constexpr int BM = 128;                 // rows per unit
 constexpr int BN = 256;                 // columns per unit
-constexpr int BK = 64;                  // tokens per pipeline stage
+#ifndef SF_DW_BK
+#define SF_DW_BK 64
+#endif
+constexpr int BK = SF_DW_BK;            // tokens per pipeline stage
 constexpr int UMMA_K = 16;              // K of one tcgen05.mma kind::f16
+static_assert(BK % UMMA_K == 0 && BK <= 256, "stage depth");
 #ifndef SF_DW_STAGES
 #define SF_DW_STAGES 4
 #endif
