@@ -57,7 +57,17 @@ constexpr int A_STAGE_BYTES = 4 * A_TILE_BYTES;    // 16 KB
 constexpr int B_BOX_BYTES = 64 * BK * 2;           // 64 columns x 64 tokens (128 B rows)
 constexpr int B_STAGE_BYTES = (BN / 64) * B_BOX_BYTES;   // 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr int TMEM_COLS = 2 * BN;       // two accumulators
+#ifndef SF_DW_NACC
+#define SF_DW_NACC 2
+#endif
+#ifndef SF_DW_CTAS_PER_SM
+#define SF_DW_CTAS_PER_SM 1
+#endif
+constexpr int NACC = SF_DW_NACC;        // TMEM accumulators per CTA (the epilogue drains one while
+                                        // the MMAs fill the other)
+constexpr int kCtasPerSm = SF_DW_CTAS_PER_SM;
+constexpr int TMEM_COLS = NACC * BN;
+static_assert(NACC * kCtasPerSm * BN <= 512, "TMEM columns per SM");
 constexpr int kThreads = 192;
 constexpr size_t kSmemBytes = (size_t)STAGES * STAGE_BYTES + 1024;   // + alignment slack
 constexpr int kMaxPerGroup = 8;
@@ -249,7 +259,7 @@ __device__ __forceinline__ Unit decode(int u, const SmemPlan &sp, const DwBatch 
 
 // ------------------------------------ main kernel ------------------------------------
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -292,7 +302,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < NACC; ++a) {
             mbar_init(&tfull_bar[a], 1);
             mbar_init(&tempty_bar[a], 4);
         }
@@ -405,7 +415,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 }
                 if (!ok) break;
                 mma_commit(&tfull_bar[acc]);
-                if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+                if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
             }
             // every MMA this thread issued has finished before TMEM is released
             mma_commit(&drain_bar);
@@ -469,7 +479,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+            if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
         }
     }
 
@@ -716,7 +726,7 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
             max_units += tiles_mt * g.n_ntiles;
         }
         if (rc != SF_OK) break;
-        const int grid = (int)(max_units < sms ? max_units : sms);
+        const int grid = (int)(max_units < (long long)sms * kCtasPerSm ? max_units : (long long)sms * kCtasPerSm);
         if (grid > 0) {
             // launches after the first of the call overlap their predecessor's last wave
             cudaLaunchAttribute attr;
