@@ -51,6 +51,8 @@ extern "C" {
 #define SF_STATUS_NONFINITE      0x2u  /* a non-finite gradient, moment or weight was produced */
 #define SF_STATUS_BAD_TOKEN      0x4u  /* a token or row id outside [0, R) was ignored */
 #define SF_STATUS_WAIT_TIMEOUT   0x8u  /* a kernel gave up a bounded wait and skipped its work */
+/* Test hook: with SF_TEST_DW_WITHHOLD=1 in the environment, sf_masked_dw's first launch withholds
+ * one pipeline stage of CTA 0, so that a bounded wait runs out and WAIT_TIMEOUT is raised. */
 
 typedef void *sf_stream;               /* cudaStream_t */
 

@@ -32,6 +32,7 @@
 //               32*(w%4)..), maps each lane to its weight row and slot, stores fp32 rows of dW.
 // Every mbarrier wait is bounded (2 s): on expiry the CTA raises SF_STATUS_WAIT_TIMEOUT, drains
 // its own TMA loads, frees its TMEM and exits.
+#include <stdlib.h>
 #include <string.h>
 
 #include "sf_common.cuh"
@@ -93,6 +94,7 @@ struct alignas(64) DwGroup {
 
 struct DwBatch {
     int32_t n_prob, n_group;
+    int32_t withhold_test;       // test hook: CTA 0 arms its first stage but issues no loads
     // variable-length payload: n_group DwGroup then n_prob DwProb
     alignas(64) unsigned char payload[32640];
 };
@@ -361,17 +363,28 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     uint8_t *sa = smem + stage * STAGE_BYTES;
                     uint8_t *sb = sa + A_STAGE_BYTES;
                     mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                    // test hook (failure detection): the stage's bytes never arrive, so the MMA
+                    // issuer's bounded wait runs out and the CTA unwinds with WAIT_TIMEOUT
+                    const bool withhold = b.withhold_test && blockIdx.x == 0 && u == (int)blockIdx.x && kb == 0;
+                    if (!withhold) {
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        if (coord[s] >= 0)
-                            tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
+                        for (int s = 0; s < 4; ++s)
+                            if (coord[s] >= 0)
+                                tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
 #pragma unroll
-                    for (int j = 0; j < BN / 64; ++j)
-                        tma_load_2d(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], x.nt * BN + j * 64, kb * BK);
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], x.nt * BN + j * 64,
+                                        kb * BK);
+                    }
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
+            }
+            {   // the MMA issuer commits drain_bar once it has finished or given up; only then is
+                // abort_flag final for this CTA
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
             }
             if (!ok || abort_flag) {
                 // drain this CTA's own loads before the shared memory goes away
@@ -604,6 +617,10 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
         if ((long long)p.mask.slot_cap * 8 > INT32_MAX) return SF_ERR_UNSUPPORTED;   // row map packing
     }
     if (n == 0) return SF_OK;
+    // Test hook for the bounded-wait path: with SF_TEST_DW_WITHHOLD set in the environment, the
+    // first main launch's CTA 0 withholds one stage of loads (see the producer).
+    const char *withhold_env = getenv("SF_TEST_DW_WITHHOLD");
+    const int withhold = withhold_env && withhold_env[0] && withhold_env[0] != '0';
     HostGroup *groups = new HostGroup[n];
     size_t need = 0;
     const int ng = plan_groups(probs, n, groups, &need);
@@ -682,6 +699,7 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
         if (g_end < ng && li + 1 >= n_launch) ++n_launch;     // an uneven split needs one more
         memset(batch, 0, sizeof(*batch));
         batch->n_group = g_end - gi;
+        batch->withhold_test = withhold && n_main_launches == 0;
         batch->n_prob = np;
         DwGroup *gd = reinterpret_cast<DwGroup *>(batch->payload);
         DwProb *pd = reinterpret_cast<DwProb *>(batch->payload + (size_t)batch->n_group * sizeof(DwGroup));

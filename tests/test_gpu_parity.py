@@ -660,3 +660,44 @@ def test_checkpoint_capacity_overflow_and_arguments(sf):
     sf.sf_mask_init(bad.mask)
     with pytest.raises(RuntimeError):
         sf.sf_checkpoint_save([sf.matrix_struct(bad)], [sf.Checkpoint(4, 24, DEV)])
+
+
+# =============================================================================================
+# failure detection: a bounded wait that runs out (no fault, no hang)
+# =============================================================================================
+
+def test_masked_dw_wait_timeout_is_reported_and_the_context_survives(sf, monkeypatch):
+    # SF_TEST_DW_WITHHOLD makes CTA 0 of the first launch arm one pipeline stage without issuing
+    # its loads. The MMA issuer's wait on that stage gives up after its limit (2 s), the CTA
+    # drains its own copies, frees its tensor memory and exits; the call reports
+    # SF_STATUS_WAIT_TIMEOUT and the next call on the same context is correct again.
+    import time
+    R, C, T = 256, 512, 512
+    words = synth.tiny_projection_mask(0, R)
+    dX = synth.normal_bf16(synth.rng(0, "dx", 9), (T, R))
+    A = synth.normal_bf16(synth.rng(0, "act", 9), (T, C))
+    mk = sf.Mask(R, R, DEV)
+    sf.sf_mask_init(mk)
+    sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_WORDS, u32_dev(words))], 0.01)
+    status = sf.status_word()
+    dW = _canary((R, C))
+    probs = [sf.dw_problem(bf16_dev(dX), bf16_dev(A), mk, dW)]
+    monkeypatch.setenv("SF_TEST_DW_WITHHOLD", "1")
+    t0 = time.perf_counter()
+    sf.sf_masked_dw(probs, status)            # tile mode (no workspace)
+    torch.cuda.synchronize()
+    took = time.perf_counter() - t0
+    assert int(host(status)[0]) & sf.SF_STATUS_WAIT_TIMEOUT
+    assert 1.5 < took < 30.0
+    monkeypatch.delenv("SF_TEST_DW_WITHHOLD")
+    status2 = sf.status_word()
+    dW2 = _canary((R, C))
+    probs2 = [sf.dw_problem(bf16_dev(dX), bf16_dev(A), mk, dW2)]
+    sf.sf_masked_dw(probs2, status2)
+    assert int(host(status2)[0]) == 0
+    ref = orc.masked_dw(dX, A, words)
+    got = host(dW2)
+    mh = mask_host(mk)
+    for r in mh["rows"]:
+        s = mh["row_slot"][r]
+        assert rel_err(got[s], ref[r]) <= DW_TOL, r
