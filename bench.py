@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense GEMM + dense Adam context line")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="skip timing the step replayed from CUDA graphs (one per input bank and coupling "
+                         "phase; the same kernels and arguments)")
     ap.add_argument("--chunks", type=int, default=1,
                     help="layer chunks per step: chunk c's masks run on a side stream while earlier "
                          "chunks' dW and update run on the main stream (1, the default and the "
@@ -741,6 +744,41 @@ def main():
     max_ms, total_rows = reduce_over_ranks(ms_total, rows_updated, device)
     value = total_rows / (max_ms / 1000.0)
 
+    graphs_out = None
+    if not args.no_graphs:
+        from masked_optimizer_step_b200.model import capture_step_graphs
+        tok_bufs = [torch.empty_like(tok_dev[0]) for _ in range(2)]
+        phases = [36.0 * j for j in range(10)]
+        graphs = [capture_step_graphs(plans[b], hp, st_ptr, tok_bufs[b], phases) for b in range(2)]
+        base = args.warmup + args.steps
+
+        def gstep(k):
+            b = k % 2
+            tok_bufs[b].copy_(tok_dev[prior + k % (tok_dev.shape[0] - prior)], non_blocking=True)
+            graphs[b][36.0 * (k % 10)].replay()
+
+        for k in range(base, base + args.warmup):
+            gstep(k)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for j, k in enumerate(range(base + args.warmup, base + args.warmup + args.steps)):
+            gstep(k)
+            counts_log[j].copy_(model.counts, non_blocking=True)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        g_rows = sum(step_work(model, c, T)["rows_updated"] for c in counts_log.cpu().numpy())
+        gms, grows = reduce_over_ranks(g0.elapsed_time(g1), g_rows, device)
+        graphs_out = {"ms_per_step": gms / args.steps, "value": grows / (gms / 1000.0),
+                      "note": "same steps replayed from CUDA graphs (20: 2 input banks x 10 coupling "
+                              "phases), token ids copied into a fixed buffer before each replay; the "
+                              "headline and the rooflines come from the un-captured timed loop"}
+        del graphs
+        for b in range(2):
+            plans[b].set_tokens(tok_dev[prior])
+
     # ---- rooflines of each stage ----
     peaks = {}
     try:
@@ -823,6 +861,8 @@ def main():
         "device_status": dev_status,
     }
 
+    if graphs_out is not None:
+        out["graphs"] = graphs_out
     if not args.no_dense and rank == 0:
         out["dense_context"] = dense_context(args.layers, T, device)
     # ---- e2e: inputs from pinned host buffers every step, result read back every step ----

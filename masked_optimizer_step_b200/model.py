@@ -320,3 +320,23 @@ class Pipeline:
             if plan.has_emb:
                 timed("embed_grad", main, lambda: plan.embed(status, sp_main))
             timed("sparse_update", main, lambda: plan.update(hp, status, sp_main))
+
+
+def capture_step_graphs(pipe: Pipeline, hp: sf.AdamParams, status, token_buf: torch.Tensor,
+                        phases_deg) -> dict:
+    """One CUDA graph of `pipe`'s step per coupling phase.
+
+    A step's kernel arguments are fixed except for two things, so a handful of graphs cover every
+    step: the token ids, read here from `token_buf` (copy each step's ids into it before replay),
+    and the pairs' coupling phase, one graph per value in `phases_deg`. The library's calls only
+    enqueue work on the given stream, so they capture as they run. Warm the calls up (run a step
+    un-captured) before capturing. Returns {phase: torch.cuda.CUDAGraph}."""
+    pipe.set_tokens(token_buf)
+    graphs = {}
+    for ph in phases_deg:
+        pipe.set_coupling(ph)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            pipe.step(hp, status, torch.cuda.current_stream())
+        graphs[ph] = g
+    return graphs

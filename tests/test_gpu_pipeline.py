@@ -18,7 +18,7 @@ SHAPES = (("q", 256, 128), ("k", 256, 128), ("v", 256, 128), ("o", 256, 128),
           ("gate", 320, 128), ("up", 320, 128), ("down", 256, 320))
 
 
-def _run(chunks):
+def _run(chunks, graphs=False):
     torch.manual_seed(0)
     model = SparseModel(3, vocab=1024, hidden=128, ffn=320, emb_slots=256, device=DEV, layer_shapes=SHAPES,
                         slot_frac=0.2)
@@ -34,10 +34,24 @@ def _run(chunks):
     hp = sf.AdamParams(device=DEV)
     status = sf.status_word(DEV)
     stream = torch.cuda.current_stream()
-    for k in range(3):
-        pipe.set_tokens(toks[k])
-        pipe.set_coupling(36.0 * k)
-        pipe.step(hp, status.data_ptr(), stream)
+    if graphs:
+        # warm the calls up un-captured on copies of nothing: one captured graph per phase,
+        # token ids copied into a fixed buffer before each replay
+        from masked_optimizer_step_b200.model import capture_step_graphs
+        buf = torch.empty_like(toks[0])
+        snap = {k: v.clone() for k, v in _state(model).items()}
+        pipe.step(hp, status.data_ptr(), stream)          # warm-up (changes state) ...
+        torch.cuda.synchronize()
+        _restore(model, snap)                              # ... so put the state back
+        g = capture_step_graphs(pipe, hp, status.data_ptr(), buf, [0.0, 36.0, 72.0])
+        for k in range(3):
+            buf.copy_(toks[k])
+            g[36.0 * k].replay()
+    else:
+        for k in range(3):
+            pipe.set_tokens(toks[k])
+            pipe.set_coupling(36.0 * k)
+            pipe.step(hp, status.data_ptr(), stream)
     torch.cuda.synchronize()
     out = []
     for m in model.all_mats:
@@ -49,6 +63,33 @@ def _run(chunks):
         rows = np.nonzero(slots >= 0)[0]
         out[-1]["moments"] = b"".join(mm[slots[r]].tobytes() + vv[slots[r]].tobytes() for r in rows)
     return out, int(host(status)[0]), len(pipe.plans)
+
+
+def _state(model):
+    """Every device array a step changes (weights, moments, gradients, mask state)."""
+    out = {}
+    for i, m in enumerate(model.all_mats):
+        for k in ("q", "s", "delta", "live", "m", "v", "grad"):
+            out[(i, k)] = getattr(m, k)
+        for k in ("charge", "accum", "words", "active_rows", "active_tiles", "tile_rows", "row_slot",
+                  "free_slots", "slot_step"):
+            out[(i, "mask." + k)] = getattr(m.mask, k)
+    out[("counts",)] = model.counts
+    return out
+
+
+def _restore(model, snap):
+    for key, t in _state(model).items():
+        t.copy_(snap[key])
+
+
+def test_step_replayed_from_cuda_graphs_matches_direct_calls(sf):
+    ref, st_ref, _ = _run(1)
+    got, st_got, _ = _run(1, graphs=True)
+    assert st_ref == st_got == 0
+    for i, (a, b) in enumerate(zip(ref, got)):
+        for key in a:
+            assert a[key] == b[key], (i, key)
 
 
 def test_chunked_schedule_matches_one_call_per_stage(sf):
