@@ -145,9 +145,13 @@ int sf_mask_update(const sf_mask *masks /* host [n_masks] */,
  * a group whose mask is scattered first gathers its active rows of dX into the scratch, so a
  * tile holds 128 active rows instead of four 32-row mask tiles; the choice is made on the device
  * from the live masks, per group, and does not change the result. With ws = NULL every group
- * runs on mask tiles. Requirements: T >= 0; C a multiple of 8; when T > 0, ld_dx and ld_a
- * multiples of 8 and dX, A 16-byte aligned; dW 16-byte aligned, ld_dw a multiple of 4 and >= C.
- * Errors: SF_ERR_ARG (also for ws smaller than needed), SF_ERR_ALIGN.
+ * runs on mask tiles. The launches of one call are chained with programmatic dependent launch:
+ * they overlap one another, never the work enqueued before or after the call. Their pipeline
+ * waits are bounded: a wait that runs out (2 s) sets SF_STATUS_WAIT_TIMEOUT and that CTA skips
+ * the rest of its work (its dW rows are then not written). Requirements: T >= 0; C a multiple of
+ * 8; when T > 0, ld_dx and ld_a multiples of 8 and dX, A 16-byte aligned; dW 16-byte aligned,
+ * ld_dw a multiple of 4 and >= C. Errors: SF_ERR_ARG (also for ws smaller than needed),
+ * SF_ERR_ALIGN, SF_ERR_UNSUPPORTED (slot_cap above 2^28).
  */
 #define SF_DW_MAX_PER_LAUNCH 96   /* problems (and groups) per launch, at most */
 
