@@ -91,3 +91,29 @@ def test_oracle_and_cuda_path_share_no_code():
             text = open(os.path.join(ROOT, "oracle", f)).read()
             assert not re.search(r"^\s*(import|from)\s+masked_optimizer_step_b200", text, re.M), f
             assert "#include" not in text or "csrc" not in text and "sf.h" not in text, f
+
+
+def test_header_is_plain_c_and_links_against_the_library(tmp_path):
+    # A C99 translation unit that takes the address of every declared entry point, compiled
+    # with gcc and linked against libsf.so (nothing runs: no GPU needed).
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    names = _declared()
+    src = ["#include \"sf.h\"", "#include <stdio.h>", "typedef void (*fn)(void);", "int main(void) {",
+           "    fn p[] = {"]
+    src += [f"        (fn){n}," for n in names]
+    src += ["    };", "    printf(\"%d %d\\n\", (int)(sizeof p / sizeof p[0]), sf_version());", "    return 0;", "}"]
+    c = tmp_path / "abi.c"
+    c.write_text("\n".join(src) + "\n")
+    lib_dir = os.path.dirname(binding.LIB_PATH)
+    out = tmp_path / "abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                        str(c), "-o", str(out), "-L", lib_dir, "-lsf", f"-Wl,-rpath,{lib_dir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(out)], capture_output=True, text=True)
+    assert run.returncode == 0, run.stderr
+    assert run.stdout.split() == [str(len(names)), str(10000)]
