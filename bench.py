@@ -69,7 +69,11 @@ def parse():
                     help="density sweep of one 11008 x 4096 projection (T = 4096), scattered and "
                          "clustered rows, with a dense bf16 GEMM and a fused dense Adam as context; "
                          "prints one JSON line per point (not the headline metric)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    args.warmup_requested = args.warmup
+    args.warmup = max(args.warmup, 3)      # at least 3 untimed warm-up steps before any timed one
+    args.steps = max(args.steps, 1)
+    return args
 
 
 def cpu_model() -> str:
