@@ -61,10 +61,12 @@ def parse():
                     help="layer chunks per step: chunk c's masks run on a side stream while earlier "
                          "chunks' dW and update run on the main stream (1, the default and the "
                          "fastest measured: one call per stage on one stream)")
-    ap.add_argument("--config", choices=["c0", "c1", "c2"], default=None,
+    ap.add_argument("--config", choices=["c0", "c1", "c2", "rewind"], default=None,
                     help="time one of the smaller workloads instead of the headline step (one JSON line "
                          "each, not the headline metric): c0 the tiny projection, c1 the embedding "
-                         "path, c2 one 7B-shaped layer at 4,096 tokens (scattered and clustered)")
+                         "path, c2 one 7B-shaped layer at 4,096 tokens (scattered and clustered), rewind "
+                         "the active-row checkpoint and a rewind-policy/Helix-driven run of the headline "
+                         "step")
     ap.add_argument("--sweep", action="store_true",
                     help="density sweep of one 11008 x 4096 projection (T = 4096), scattered and "
                          "clustered rows, with a dense bf16 GEMM and a fused dense Adam as context; "
@@ -569,6 +571,112 @@ def _stage_line(model, pipe, hp, status, T, steps, warm, stream, before_step=Non
     return t0.elapsed_time(t1) / steps, st / steps, work
 
 
+def run_rewind(args):
+    """Active-row checkpoint and rewind at the headline shape: save and restore of every matrix's
+    active rows timed with CUDA events against their algorithmic bytes, then a run of the step
+    driven by the rewind policy and the Helix coupling schedule on a synthetic loss curve with one
+    planted rebound (the policy saves, watches, rewinds and skips as it would in training)."""
+    import torch
+    from masked_optimizer_step_b200 import binding as sf
+    from masked_optimizer_step_b200 import helix as hx
+    from masked_optimizer_step_b200.model import Pipeline, SparseModel
+    sf.load()
+    device = "cuda:0"
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    T = args.tokens
+    model = SparseModel(n_layers=args.layers, device=device)
+    model.init(SEED)
+    banks = [make_bank(model, T, args.masks, b, device) for b in range(2)]
+    prior, n_run = 20, 60
+    toks = torch.from_numpy(token_stream(prior + n_run + 3, T)).to(device)
+    for b in banks:
+        b["tokens"] = toks[prior]
+    ws = torch.zeros(sf.sf_embed_grad_ws_bytes(T, model.emb.mask.slot_cap) // 4 + 64, dtype=torch.int32,
+                     device=device)
+    pipes = [Pipeline(model, b, ws) for b in banks]
+    hp = sf.AdamParams(device=device)
+    status = sf.status_word(device)
+    st_ptr = status.data_ptr()
+    for w in range(prior):
+        sf.sf_mask_update([model.emb.mask], [sf.make_src(sf.SF_SRC_TOKENS, toks[w], n=T)], 0.01, status)
+    for k in range(3):                                       # warm-up steps: masks and slots settle
+        pipes[k % 2].set_tokens(toks[prior + k])
+        pipes[k % 2].step(hp, st_ptr, stream)
+    torch.cuda.synchronize()
+    helix = hx.Helix()
+    rw = hx.Rewinder(model.all_mats, hx.RewindPolicy(), helix, device=device)
+    counts = model.counts.cpu().numpy()
+    rows = int(sum(min(int(c[0]), m.mask.slot_cap) for c, m in zip(counts, model.all_mats)))
+    row_bytes = sum(min(int(c[0]), m.mask.slot_cap) * (9 * m.C + 12) for c, m in zip(counts, model.all_mats))
+    live_bytes = sum(min(int(c[0]), m.mask.slot_cap) * 2 * m.C for c, m in zip(counts, model.all_mats))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    save_ms = timed(lambda: rw.save(st_ptr, stream.cuda_stream))
+    restore_ms = timed(lambda: rw.restore(st_ptr, stream.cuda_stream))
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    save_gbs = 2 * row_bytes / (save_ms / 1e3) / 1e9
+    restore_gbs = (2 * row_bytes + live_bytes) / (restore_ms / 1e3) / 1e9
+
+    # the policy- and schedule-driven run: the loss falls, then rebounds by 60% from step 30 on,
+    # so each watch that ends during the rebound rewinds (at most three times per minimum)
+    g = np.random.default_rng(SEED)
+    losses = [2.0 * math.exp(-k / 25.0) + 0.6 + 0.004 * g.standard_normal() for k in range(n_run)]
+    for k in range(30, n_run):
+        losses[k] *= 1.6
+    rw.policy = hx.RewindPolicy()
+    rw.saved = False
+    events, stride_seen = {}, []
+    e0.record(stream)
+    done = 0
+    for k in range(n_run):
+        pipe = pipes[k % 2]
+        act = rw.before_step(losses[k - 1] if k else losses[0], st_ptr, stream.cuda_stream)
+        events[act.event or "step"] = events.get(act.event or "step", 0) + 1
+        stride_seen.append(helix.stride.value)
+        if act.skip:
+            continue
+        c = helix.coefficients()
+        pipe.set_mix(c.c_self, c.c_partner)
+        pipe.set_tokens(toks[prior + 3 + k])
+        pipe.step(hp, st_ptr, stream)
+        done += 1
+    e1.record(stream)
+    torch.cuda.synchronize()
+    run_ms = e0.elapsed_time(e1)
+    line = {"config": "rewind",
+            "workload": f"checkpoint and rewind of the active rows of the {args.layers}-layer 7B-shaped step "
+                        f"({args.tokens} tokens, ~1% {args.masks} rows); policy + Helix run of {n_run} steps on a "
+                        "synthetic loss curve with a planted 60% rebound from step 30",
+            "checkpoint": {"rows": rows, "matrices": len(model.all_mats),
+                           "save_ms": save_ms, "restore_ms": restore_ms,
+                           "save_gbs": save_gbs, "restore_gbs": restore_gbs,
+                           "save_frac_hbm": save_gbs / hbm, "restore_frac_hbm": restore_gbs / hbm,
+                           "algorithmic": "9*C+12 B per saved row each way (q, delta, m, v, s, step, row id); "
+                                          "restore also writes the bf16 live row"},
+            "policy_run": {"steps": n_run, "steps_applied": done, "ms_total": run_ms,
+                           "ms_per_applied_step": run_ms / max(done, 1), "events": events,
+                           "max_stride": max(stride_seen), "final_phase_deg": helix.phi_deg % 360.0},
+            "device_status": int(status.cpu()[0])}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_config(args):
     """The smaller workloads: c0 the tiny projection (256 x 512, 128 tokens, fixed 3%-row mask,
     3 Adam steps), c1 the embedding path (32,000 x 4,096 table, 8 x 512 Zipf(1.1) tokens, seed 1,
@@ -668,6 +776,8 @@ def main():
         return run_reference(args)
     if args.sweep:
         return run_sweep(args)
+    if args.config == "rewind":
+        return run_rewind(args)
     if args.config:
         return run_config(args)
     rank, world, local = dist_env()

@@ -335,21 +335,42 @@ class Rewinder:
         self.ckpts = [sf.Checkpoint(m.mask.slot_cap if m.mask.slot_cap else m.R, m.C, device)
                       for m in self.mats]
         self.saved = False
+        self._args = None                  # ctypes argument arrays, built once (pointers are fixed)
 
     def structs(self):
         return [self.sf.matrix_struct(m) for m in self.mats]
 
+    def _call(self, name, status, stream):
+        sf = self.sf
+        if not hasattr(sf, "load"):        # a stand-in binding (host tests): plain calls
+            getattr(sf, name)(self.structs(), self.ckpts, status, stream)
+            return
+        if getattr(self, "_args", None) is None:
+            n = len(self.mats)
+            self._args = ((sf.sf_matrix * n)(*self.structs()),
+                          (sf.sf_checkpoint * n)(*[c.struct() for c in self.ckpts]), n)
+        mats, cks, n = self._args
+        st = status if status is None or isinstance(status, int) else status.data_ptr()
+        sm = stream if stream is None or isinstance(stream, int) else stream.cuda_stream
+        sf._check(getattr(sf.load(), name)(mats, cks, n, st, sm), name)
+
+    def save(self, status=None, stream=None):
+        self._call("sf_checkpoint_save", status, stream)
+        self.saved = True
+
+    def restore(self, status=None, stream=None):
+        self._call("sf_checkpoint_restore", status, stream)
+
     def before_step(self, loss: float, status=None, stream=None) -> Action:
         act = self.policy.observe(loss)
         if act.restore and self.saved:
-            self.sf.sf_checkpoint_restore(self.structs(), self.ckpts, status, stream)
+            self.restore(status, stream)
             if self.helix is not None:
                 self.helix.rewind()
         elif act.restore:
             act = Action(event="")
         if act.save:
-            self.sf.sf_checkpoint_save(self.structs(), self.ckpts, status, stream)
-            self.saved = True
+            self.save(status, stream)
         if self.helix is not None and not act.skip:
             self.helix.push_loss(loss)
         return act
