@@ -42,7 +42,13 @@ namespace sf {
 namespace {
 
 constexpr int BM = 128;                 // rows per unit
-constexpr int BN = 256;                 // columns per unit
+#ifndef SF_DW_BN
+#define SF_DW_BN 256
+#endif
+constexpr int BN = SF_DW_BN;            // columns per unit
+constexpr int MMA_N = BN > 256 ? 256 : BN;   // N of one tcgen05.mma (at most 256)
+constexpr int NSUB = BN / MMA_N;             // MMAs per 16-token step across the unit's columns
+static_assert(BN % MMA_N == 0 && MMA_N % 64 == 0, "column tiling");
 #ifndef SF_DW_BK
 #define SF_DW_BK 64
 #endif
@@ -150,7 +156,7 @@ constexpr uint32_t kLayoutSW64 = 4;
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both MN-major, N, M.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+                            ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 // Row mode when the group's active rows fit the scratch and need fewer 128-row tiles than the
 // mask tiles do. Every reader computes the same answer from the same counts.
@@ -420,8 +426,12 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // 16 tokens = 16 rows of 64 B (A-operand) or 128 B (B-operand)
                         const uint64_t da = smem_desc(sa + k * UMMA_K * 64, A_TILE_BYTES, 8 * 64, kLayoutSW64);
-                        const uint64_t db = smem_desc(sb + k * UMMA_K * 128, B_BOX_BYTES, 8 * 128, kLayoutSW128);
-                        mma_bf16(d_tmem, da, db, kIdesc, (kb | k) != 0);
+#pragma unroll
+                        for (int h = 0; h < NSUB; ++h) {
+                            const uint64_t db = smem_desc(sb + h * (MMA_N / 64) * B_BOX_BYTES + k * UMMA_K * 128,
+                                                          B_BOX_BYTES, 8 * 128, kLayoutSW128);
+                            mma_bf16(d_tmem + h * MMA_N, da, db, kIdesc, (kb | k) != 0);
+                        }
                     }
                     mma_commit(&empty_bar[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
