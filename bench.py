@@ -34,8 +34,8 @@ METRIC = "sparse step ms & active-row updates/s at 7B shape, 1% active; % of roo
 # DRAM traffic per layer of each stage (dram__bytes_read.sum + dram__bytes_write.sum), measured
 # with ncu on the 2-layer case of the default workload (scattered masks, 2,048 tokens) and
 # scaled by the layer count; it applies to that workload only.
-TRAFFIC_PER_LAYER = {"masks": (348.588e6 + 3.606e6 + 1.446e6 + 0.000e6) / 2,               # accumulate + finalize
-                     "masked_dw": (173.731e6 + 3.483e6 + 204.449e6 + 7.895e6) / 2}    # gather + main
+TRAFFIC_PER_LAYER = {"masks": (348.541e6 + 3.842e6 + 1.447e6 + 0.000e6) / 2,               # accumulate + finalize
+                     "masked_dw": (173.725e6 + 3.578e6 + 204.643e6 + 8.520e6) / 2}    # gather + main
 UNIT = "active-row updates/s"
 SEED = 3
 SWEEP_SEED = 4
