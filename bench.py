@@ -639,26 +639,22 @@ def run_rewind(args):
     losses = [2.0 * math.exp(-k / 25.0) + 0.6 + 0.004 * g.standard_normal() for k in range(n_run)]
     for k in range(30, n_run):
         losses[k] *= 1.6
-    rw.policy = hx.RewindPolicy()
-    rw.saved = False
-    events, stride_seen = {}, []
+    from masked_optimizer_step_b200.model import Trainer
+    del rw                                                   # its checkpoint buffers
+    torch.cuda.empty_cache()
+    trainer = Trainer(model, pipes, hp, status, stream)
+    helix = trainer.helix
+    stride_seen = []
     e0.record(stream)
     done = 0
     for k in range(n_run):
-        pipe = pipes[k % 2]
-        act = rw.before_step(losses[k - 1] if k else losses[0], st_ptr, stream.cuda_stream)
-        events[act.event or "step"] = events.get(act.event or "step", 0) + 1
+        act = trainer.step(k, losses[k - 1] if k else losses[0], tokens=toks[prior + 3 + k])
         stride_seen.append(helix.stride.value)
-        if act.skip:
-            continue
-        c = helix.coefficients()
-        pipe.set_mix(c.c_self, c.c_partner)
-        pipe.set_tokens(toks[prior + 3 + k])
-        pipe.step(hp, st_ptr, stream)
-        done += 1
+        done += not act.skip
     e1.record(stream)
     torch.cuda.synchronize()
     run_ms = e0.elapsed_time(e1)
+    events = trainer.events
     line = {"config": "rewind",
             "workload": f"checkpoint and rewind of the active rows of the {args.layers}-layer 7B-shaped step "
                         f"({args.tokens} tokens, ~1% {args.masks} rows); policy + Helix run of {n_run} steps on a "

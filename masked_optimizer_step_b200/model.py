@@ -340,3 +340,38 @@ def capture_step_graphs(pipe: Pipeline, hp: sf.AdamParams, status, token_buf: to
             pipe.step(hp, status, torch.cuda.current_stream())
         graphs[ph] = g
     return graphs
+
+
+class Trainer:
+    """The host loop around the step ("Sparse-First Fine-Tuning", sections 2.4-2.6).
+
+    Each call to `step` takes the loss of the previous step (read after that step, so nothing is
+    read back in the middle of one), lets the rewind policy save or restore the active-row
+    checkpoint, sets every pair's mix from the Helix schedule, and issues the step on `stream`,
+    or skips it when the policy has just rewound. `pipes` are Pipeline objects over the same
+    model (e.g. one per input bank); step k uses pipes[k % len(pipes)]."""
+
+    def __init__(self, model: SparseModel, pipes, hp: sf.AdamParams, status, stream=None,
+                 policy=None, helix=None, device=None):
+        from . import helix as hx
+        self.model, self.pipes, self.hp, self.status = model, list(pipes), hp, status
+        self.stream = stream
+        self.helix = helix if helix is not None else hx.Helix()
+        self.rewinder = hx.Rewinder(model.all_mats, policy or hx.RewindPolicy(), self.helix,
+                                    device=device or model.device)
+        self.events = {}
+
+    def step(self, k: int, prev_loss: float, tokens: torch.Tensor | None = None):
+        stream = self.stream if self.stream is not None else torch.cuda.current_stream()
+        st = self.status.data_ptr() if hasattr(self.status, "data_ptr") else self.status
+        act = self.rewinder.before_step(prev_loss, st, stream.cuda_stream)
+        self.events[act.event or "step"] = self.events.get(act.event or "step", 0) + 1
+        if act.skip:
+            return act
+        pipe = self.pipes[k % len(self.pipes)]
+        c = self.helix.coefficients()
+        pipe.set_mix(c.c_self, c.c_partner)
+        if tokens is not None:
+            pipe.set_tokens(tokens)
+        pipe.step(self.hp, st, stream)
+        return act

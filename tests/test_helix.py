@@ -302,3 +302,44 @@ def test_rewinder_drives_save_and_restore_and_resets_the_stride():
     a = rw.before_step(2.7)                    # 2.7 > 1.15 * 2.3
     assert a.skip and fake.calls[-1] == ("restore", 2)
     assert rw.helix.stride.value == 1
+
+
+class _FakePipe:
+    def __init__(self, log, name):
+        self.log, self.name = log, name
+
+    def set_mix(self, c_self, c_partner):
+        self.log.append((self.name, "mix", round(c_partner["gate-up"], 6)))
+
+    def set_tokens(self, t):
+        self.log.append((self.name, "tokens", t))
+
+    def step(self, hp, status, stream):
+        self.log.append((self.name, "step"))
+
+
+def test_trainer_orders_policy_mix_and_step_and_skips_after_a_rewind():
+    from masked_optimizer_step_b200.model import Trainer
+    fake = _FakeBinding()
+    rw = hx.Rewinder.__new__(hx.Rewinder)
+    rw.sf, rw.mats = fake, [_FakeMat(64, 32, 8)]
+    rw.policy, rw.helix, rw.saved = hx.RewindPolicy(), hx.Helix(), False
+    rw.ckpts = [fake.Checkpoint(8, 32, "cpu")]
+    log = []
+    tr = Trainer.__new__(Trainer)
+    tr.model, tr.pipes, tr.hp, tr.status = None, [_FakePipe(log, "a"), _FakePipe(log, "b")], None, 0
+    tr.stream = type("S", (), {"cuda_stream": 0})()
+    tr.helix, tr.rewinder, tr.events = rw.helix, rw, {}
+    losses = [2.0, 1.95, 1.9] + [2.3] * 10                 # 2.3 > 1.15 * 1.9: the watch ends in a rewind
+    acts = [tr.step(k, L, tokens=k) for k, L in enumerate(losses)]
+    assert [a.event for a in acts[:3]] == ["watch"] * 3
+    assert acts[12].skip and acts[12].event == "rewind" and fake.calls[-1] == ("restore", 1)
+    steps = [e for e in log if e[1] == "step"]
+    assert len(steps) == 12                                  # every step but the rewound one
+    assert steps[0][0] == "a" and steps[1][0] == "b"       # pipes alternate by step index
+    # before each step: the mix, then the tokens, then the step, on the same pipe
+    for i, e in enumerate(log):
+        if e[1] == "step":
+            assert log[i - 1][0] == e[0] and log[i - 1][1] == "tokens"
+            assert log[i - 2][0] == e[0] and log[i - 2][1] == "mix"
+    assert tr.events["rewind"] == 1 and rw.helix.stride.value == 1
