@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--no-graphs", action="store_true",
                     help="skip timing the step replayed from CUDA graphs (one per input bank and coupling "
                          "phase; the same kernels and arguments)")
+    ap.add_argument("--no-overlap-embedding", action="store_true",
+                    help="keep the embedding's conductor and row gradient on the main stream (by default "
+                         "they run on a side stream, concurrent with the projections' trackers and dW)")
     ap.add_argument("--chunks", type=int, default=1,
                     help="layer chunks per step: chunk c's masks run on a side stream while earlier "
                          "chunks' dW and update run on the main stream (1, the default and the "
@@ -117,8 +120,10 @@ def workload_config(args):
         "hidden": 4096, "ffn": 11008, "vocab": 32000,
         "l2": "no flush needed: each step reads ~14 GB of resident inputs (L2 is 126 MB)",
         "parallelism": "replicas",
-        "schedule": f"{args.chunks} layer chunks, masks on a side stream overlapping earlier chunks' dW and update"
-                    if args.chunks > 1 else "one call per stage, one stream",
+        "schedule": (f"{args.chunks} layer chunks, masks on a side stream overlapping earlier chunks' dW and update"
+                     if args.chunks > 1 else
+                     "one call per stage; the embedding's conductor and row gradient on a side stream"
+                     if not args.no_overlap_embedding else "one call per stage, one stream"),
     }
 
 
@@ -801,7 +806,8 @@ def main():
         b["tokens"] = tok_dev[prior]
     ws = torch.zeros(sf.sf_embed_grad_ws_bytes(T, model.emb.mask.slot_cap) // 4 + 64, dtype=torch.int32,
                      device=device)
-    plans = [Pipeline(model, b, ws, chunks=args.chunks) for b in banks]
+    plans = [Pipeline(model, b, ws, chunks=args.chunks, overlap_embedding=not args.no_overlap_embedding)
+             for b in banks]
     hp = sf.AdamParams(device=device)
     status = sf.status_word(device)
     stream = torch.cuda.current_stream()
@@ -842,8 +848,8 @@ def main():
     if world > 1:
         dist.barrier()
     ms_total = t_start.elapsed_time(t_end)
-    stage_names = ("masks", "masked_dw", "embed_grad", "sparse_update")
-    stage_ms = np.zeros(4)
+    stage_names = ("masks", "masked_dw", "embed_grad", "sparse_update", "conductor")
+    stage_ms = np.zeros(5)
     for name, e0, e1 in timing:
         stage_ms[stage_names.index(name)] += e0.elapsed_time(e1)
     counts = counts_log.cpu().numpy()
@@ -927,7 +933,12 @@ def main():
         "masks": {"ms_per_step": stage_ms[0] / args.steps, "bound": "hbm", "achieved": trk_gbs,
                   "peak": hbm, "unit": "GB/s", "frac": trk_gbs / hbm, "algorithmic": "Y read once: T*R*2 B per projection"},
         "masked_dw": dw_stage,
-        "embed_grad": {"ms_per_step": stage_ms[2] / args.steps},
+        "embed_grad": {"ms_per_step": stage_ms[2] / args.steps,
+                       "stream": "side (overlapped)" if not args.no_overlap_embedding else "main"},
+        "conductor": {"ms_per_step": stage_ms[4] / args.steps, "stream": "side (overlapped)",
+                      "note": "the embedding's mask, its own call concurrent with the trackers; its "
+                              "event-timed span includes waiting for SMs"} if not args.no_overlap_embedding
+                     else {"ms_per_step": 0.0, "note": "part of the masks call"},
         "sparse_update": {"ms_per_step": stage_ms[3] / args.steps, "bound": "hbm", "achieved": upd_gbs,
                           "peak": hbm, "unit": "GB/s", "frac": upd_gbs / hbm,
                           "algorithmic": "24 B per active element (20 on fresh rows) + 8 B per row"},

@@ -160,6 +160,9 @@ class StepPlan:
             Y = inputs["Y"][i]
             srcs.append(sf.sf_mask_src(sf.SF_SRC_OUTPUT_BF16, Y.shape[0], Y.stride(0), Y.data_ptr()))
         self.src_arr = (sf.sf_mask_src * n)(*srcs)
+        off = 1 if self.has_emb else 0             # the trackers alone, for a split masks stage
+        self.proj_mask_arr = (sf.sf_mask * max(n - off, 1))(*[m.mask.struct() for m in mats[off:]])
+        self.proj_src_arr = (sf.sf_mask_src * max(n - off, 1))(*srcs[off:])
         probs = [sf.dw_problem(inputs["dX"][i], inputs["A"][i], p.mat.mask, p.mat.grad).c for i, p in projs]
         self.n_dw = len(probs)
         self.dw_arr = (sf.sf_dw_problem * max(len(probs), 1))(*probs)
@@ -205,6 +208,22 @@ class StepPlan:
             self.upd_arr[k + off].c_partner = c_partner.get(pair, 0.0) if pair else 0.0
 
     # the four calls of one step --------------------------------------------------------------
+    def masks_embedding(self, status, stream):
+        """The conductor alone (the embedding's mask), as its own call."""
+        if not self.has_emb:
+            return
+        sf._check(self.lib.sf_mask_update(self.mask_arr, self.src_arr, 1, self.threshold, status, stream),
+                  "sf_mask_update")
+
+    def masks_projections(self, status, stream):
+        """The row trackers of every projection of the plan, as one call."""
+        off = 1 if self.has_emb else 0
+        n = self.n_masks - off
+        if n <= 0:
+            return
+        sf._check(self.lib.sf_mask_update(self.proj_mask_arr, self.proj_src_arr, n, self.threshold, status,
+                                          stream), "sf_mask_update")
+
     def masks(self, status, stream):
         sf._check(self.lib.sf_mask_update(self.mask_arr, self.src_arr, self.n_masks, self.threshold,
                                           status, stream), "sf_mask_update")
@@ -230,12 +249,14 @@ class StepPlan:
         sf._check(self.lib.sf_sparse_update(self.upd_arr, len(self.upd_arr), ctypes.byref(h), status,
                                             stream), "sf_sparse_update")
 
-    def launches(self) -> int:
+    def launches(self, split_embedding: bool = False) -> int:
         """Kernel launches one step issues (for the launch count of a timed region)."""
         def chunks(n, k):
             return (n + k - 1) // k
-        n_mask_batches = chunks(self.n_masks, sf.SF_MASKS_PER_LAUNCH)
-        n = 2 * n_mask_batches                       # accumulate + finalize per batch of masks
+        if split_embedding and self.has_emb:         # conductor and trackers as two calls
+            n = 2 + 2 * chunks(self.n_masks - 1, sf.SF_MASKS_PER_LAUNCH) if self.n_masks > 1 else 2
+        else:
+            n = 2 * chunks(self.n_masks, sf.SF_MASKS_PER_LAUNCH)   # accumulate + finalize per batch
         n += 2 * self.dw_launches                   # gather + main kernel per launch
         n += 2 if self.has_emb else 0
         n += chunks(len(self.upd_arr), sf.SF_MATS_PER_LAUNCH)
@@ -256,7 +277,8 @@ class Pipeline:
     kernel's persistent CTAs take their units by index, so CTAs that the concurrent tracker pass
     keeps off the SMs start late and stretch the launch, and both streams draw on the same HBM."""
 
-    def __init__(self, model: SparseModel, inputs: dict, embed_ws, chunks: int = 4, threshold: float = 0.01):
+    def __init__(self, model: SparseModel, inputs: dict, embed_ws, chunks: int = 4, threshold: float = 0.01,
+                 overlap_embedding: bool = False):
         layers = sorted({p.layer for p in model.projs})
         chunks = max(1, min(chunks, len(layers))) if layers else 1
         bounds = [0]
@@ -271,6 +293,10 @@ class Pipeline:
         self.side = torch.cuda.Stream(device=model.device)
         self.start = torch.cuda.Event()
         self.masks_done = [torch.cuda.Event() for _ in self.plans]
+        # one call per stage, but the embedding's conductor and row gradient on the side stream,
+        # concurrent with the projections' trackers and dW; joined before the update
+        self.overlap_embedding = overlap_embedding and len(self.plans) == 1 and self.plans[0].has_emb
+        self.emb_done = torch.cuda.Event()
 
     def set_tokens(self, tokens):
         self.plans[0].set_tokens(tokens)
@@ -284,7 +310,7 @@ class Pipeline:
             p.set_mix(c_self, c_partner)
 
     def launches(self) -> int:
-        return sum(p.launches() for p in self.plans)
+        return sum(p.launches(self.overlap_embedding) for p in self.plans)
 
     def step(self, hp: sf.AdamParams, status, main, timing: list | None = None):
         """Issue one step. main: the torch stream the step belongs to; timing: if a list, gets
@@ -302,6 +328,18 @@ class Pipeline:
             e1.record(stream)
             timing.append((stage, e0, e1))
 
+        if self.overlap_embedding:
+            plan = self.plans[0]
+            self.start.record(main)
+            side.wait_event(self.start)
+            timed("conductor", side, lambda: plan.masks_embedding(status, sp_side))
+            timed("embed_grad", side, lambda: plan.embed(status, sp_side))
+            self.emb_done.record(side)
+            timed("masks", main, lambda: plan.masks_projections(status, sp_main))
+            timed("masked_dw", main, lambda: plan.dw(status, sp_main))
+            main.wait_event(self.emb_done)
+            timed("sparse_update", main, lambda: plan.update(hp, status, sp_main))
+            return
         if len(self.plans) == 1:                     # one call per stage, all on the main stream
             plan = self.plans[0]
             timed("masks", main, lambda: plan.masks(status, sp_main))

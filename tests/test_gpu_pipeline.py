@@ -18,7 +18,7 @@ SHAPES = (("q", 256, 128), ("k", 256, 128), ("v", 256, 128), ("o", 256, 128),
           ("gate", 320, 128), ("up", 320, 128), ("down", 256, 320))
 
 
-def _run(chunks, graphs=False):
+def _run(chunks, graphs=False, overlap=False):
     torch.manual_seed(0)
     model = SparseModel(3, vocab=1024, hidden=128, ffn=320, emb_slots=256, device=DEV, layer_shapes=SHAPES,
                         slot_frac=0.2)
@@ -30,7 +30,7 @@ def _run(chunks, graphs=False):
     bank["tokens"] = toks[0]
     ws = torch.zeros(sf.sf_embed_grad_ws_bytes(T, model.emb.mask.slot_cap) // 4 + 64, dtype=torch.int32,
                      device=DEV)
-    pipe = Pipeline(model, bank, ws, chunks=chunks)
+    pipe = Pipeline(model, bank, ws, chunks=chunks, overlap_embedding=overlap)
     hp = sf.AdamParams(device=DEV)
     status = sf.status_word(DEV)
     stream = torch.cuda.current_stream()
@@ -98,6 +98,24 @@ def test_chunked_schedule_matches_one_call_per_stage(sf):
     assert n1 == 1 and n3 == 3
     assert st_ref == st_got == 0
     assert len(ref) == len(got)
+    for i, (a, b) in enumerate(zip(ref, got)):
+        for key in a:
+            assert a[key] == b[key], (i, key)
+
+
+def test_embedding_on_a_side_stream_matches_one_call_per_stage(sf):
+    ref, st_ref, _ = _run(1)
+    got, st_got, _ = _run(1, overlap=True)
+    assert st_ref == st_got == 0
+    for i, (a, b) in enumerate(zip(ref, got)):
+        for key in a:
+            assert a[key] == b[key], (i, key)
+
+
+def test_embedding_overlap_replayed_from_graphs_matches(sf):
+    ref, _, _ = _run(1)
+    got, st_got, _ = _run(1, graphs=True, overlap=True)
+    assert st_got == 0
     for i, (a, b) in enumerate(zip(ref, got)):
         for key in a:
             assert a[key] == b[key], (i, key)
