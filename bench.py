@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense GEMM + dense Adam context line")
+    ap.add_argument("--step-log", default=None, metavar="PATH",
+                    help="write one JSON line per timed step: ms per call, active rows (total and per "
+                         "matrix), active tiles, rows without a slot, fresh slots, dW row-mode groups")
     ap.add_argument("--no-graphs", action="store_true",
                     help="skip timing the step replayed from CUDA graphs (one per input bank and coupling "
                          "phase; the same kernels and arguments)")
@@ -839,8 +842,10 @@ def main():
     clocks.start()
     time.sleep(0.1)
     t_start.record(stream)
+    step_marks = []
     for k in range(args.steps):
         step(args.warmup + k, timing)
+        step_marks.append(len(timing))
         counts_log[k].copy_(model.counts, non_blocking=True)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -856,6 +861,23 @@ def main():
     work = [step_work(model, counts[k], T) for k in range(args.steps)]
     rows_updated = sum(w["rows_updated"] for w in work)
     dev_status = int(status.cpu()[0])
+    if args.step_log and rank == 0:
+        names = ["embedding"] + [f"L{p.layer}.{p.name}" for p in model.projs]
+        with open(args.step_log, "w") as f:
+            lo = 0
+            for k, hi in enumerate(step_marks):
+                calls = {}
+                for name, e0, e1 in timing[lo:hi]:
+                    calls[name] = calls.get(name, 0.0) + e0.elapsed_time(e1)
+                lo = hi
+                c = counts[k]
+                f.write(json.dumps({
+                    "step": args.warmup + k, "ms_per_call": calls,
+                    "active_rows": int(c[:, 0].sum()), "active_tiles": int(c[1:, 1].sum()),
+                    "rows_without_slot": int(c[:, 3].sum()), "fresh_slots": int(c[:, 4].sum()),
+                    "rows_updated": work[k]["rows_updated"], "dw_row_mode_groups": work[k]["dw_row_groups"],
+                    "update_mb": work[k]["update_bytes"] / 1e6,
+                    "active_rows_per_matrix": dict(zip(names, (int(x) for x in c[:, 0])))}) + "\n")
 
     max_ms, total_rows = reduce_over_ranks(ms_total, rows_updated, device)
     value = total_rows / (max_ms / 1000.0)
