@@ -125,6 +125,26 @@ def dw_launch_count(problems, group_bytes=320, prob_bytes=192, payload=32640, ma
     return launches
 
 
+def dw_gather_launch_count(problems, max_groups=192, max_probs=384, max_per_group=8) -> int:
+    """Launches of the row gather that sf_masked_dw issues when given a workspace: the call's
+    groups (consecutive problems reading the same input, at most max_per_group) packed in order
+    into launches of at most max_groups groups and max_probs problems. problems: [(input, C)]."""
+    groups = []
+    for key in problems:
+        if groups and groups[-1][0] == key and groups[-1][1] < max_per_group:
+            groups[-1][1] += 1
+        else:
+            groups.append([key, 1])
+    launches, ng, npb = 0, 0, 0
+    for _, cnt in groups:
+        if ng == 0 or ng >= max_groups or npb + cnt > max_probs:
+            launches += 1
+            ng, npb = 0, 0
+        ng += 1
+        npb += cnt
+    return launches
+
+
 class StepPlan:
     """ABI argument arrays of one step over `model` for one set of input buffers.
 
@@ -180,7 +200,9 @@ class StepPlan:
             structs.append(sf.matrix_struct(p.mat, g, 1.0, 0.0))
         self.upd_arr = (sf.sf_matrix * len(structs))(*structs)
         self.embed_ws = embed_ws
-        self.dw_launches = dw_launch_count([(id(inputs["A"][i]), p.mat.C) for i, p in projs]) if projs else 0
+        keys = [(id(inputs["A"][i]), p.mat.C) for i, p in projs]
+        self.dw_launches = dw_launch_count(keys) if projs else 0
+        self.gather_launches = dw_gather_launch_count(keys) if projs else 0
         if self.has_emb:
             self.emb_mask = model.emb.mask.struct()
 
@@ -257,7 +279,7 @@ class StepPlan:
             n = 2 + 2 * chunks(self.n_masks - 1, sf.SF_MASKS_PER_LAUNCH) if self.n_masks > 1 else 2
         else:
             n = 2 * chunks(self.n_masks, sf.SF_MASKS_PER_LAUNCH)   # accumulate + finalize per batch
-        n += 2 * self.dw_launches                   # gather + main kernel per launch
+        n += self.gather_launches + self.dw_launches  # row gather, then the main dW launches
         n += 2 if self.has_emb else 0
         n += chunks(len(self.upd_arr), sf.SF_MATS_PER_LAUNCH)
         return n
