@@ -174,10 +174,12 @@ int sf_masked_dw(const sf_dw_problem *probs /* host [n] */, int n, void *ws, siz
 
 /* ---- sf_embed_grad: sections 1 and 2.2 (embedding rows) ---------------------------------
  * A row's gradient comes only from the batch positions holding its token, and only rows the
- * mask marks active are computed: for each active row r with slot k,   G[k * ld_g + c] = sum over tokens t with tokens[t] == r of dY[t, c]
+ * mask marks active are computed: for each active row r with slot k,
+ *     G[k * ld_g + c] = sum over tokens t with tokens[t] == r of dY[t, c]
  * (fp32; an active row with no token gets zeros). dY is [n_tok x ld_dy] bf16, H columns.
  * Tokens of inactive rows are dropped. Deterministic: each row's tokens are summed in one fixed
- * order. Needs caller scratch `ws` of sf_embed_grad_ws_bytes() bytes (16-byte aligned).
+ * order (ascending position, split over eight partial sums that are added in a fixed order).
+ * Needs caller scratch `ws` of sf_embed_grad_ws_bytes() bytes (16-byte aligned).
  * Limits: n_tok <= 16384, slot_cap <= 49152 (SF_ERR_UNSUPPORTED beyond).
  * Requirements: H, ld_dy multiples of 8, ld_g multiple of 4 >= H, dY and G 16-byte aligned.
  */
@@ -195,8 +197,9 @@ int sf_embed_grad(const int32_t *tokens, int n_tok, const void *dY, int H, int64
  * is a fixed array of SF_EMBED_NOALLOC_SCRATCH_INTS int32 (256 KiB) in the library's own device
  * memory, present on every GPU that loads the library until the process exits; a call needs
  * slot_cap + 1 + n_tok of them and returns SF_ERR_UNSUPPORTED beyond that. The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) and caches it; make that
- * first call before any stream capture. All calls on a GPU share the array: calls that can
+ * device looks up the array's device address (cudaGetSymbolAddress) and caches it for the
+ * device's current context (a new context, e.g. after cudaDeviceReset, repeats the lookup); make
+ * that first call before any stream capture. All calls on a GPU share the array: calls that can
  * overlap on the GPU (different streams or threads) race on it and must be ordered by the
  * caller. This entry point allocates nothing.
  */

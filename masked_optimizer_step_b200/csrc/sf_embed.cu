@@ -6,18 +6,23 @@
 // upstream gradients dY[t] over the batch positions t holding token r, and only rows the
 // conductor marks active are computed and stored.
 //
-// Two launches:
+// Three launches:
 //   embed_index_kernel  one CTA: for every token whose row is active, its slot; per-slot counts
 //                       (shared-memory atomics, exact), an exclusive scan into segment offsets,
 //                       and a scatter of token positions into their slot's segment of ws.
-//   embed_sum_kernel    persistent: one item = (active row, 256-column chunk). The CTA loads its
-//                       row's segment, sorts the positions ascending (rank sort in shared
-//                       memory, so the sum order never depends on atomics), then 8 warps each
-//                       sum every 8th token of the segment with 16-byte loads and the partial
-//                       sums are added in warp order. Active rows without tokens get zeros.
+//   embed_sort_kernel   one CTA per active row at a time: the row's segment is sorted ascending
+//                       in shared memory (bitonic network), once per row, so the sum order
+//                       never depends on the order the scatter's atomics happened to take.
+//   embed_sum_kernel    persistent: one item = (active row, 256-column chunk). 8 warps each
+//                       sum every 8th token of the row's sorted segment with 16-byte loads (eight
+//                       in flight per lane) and the partial sums are added in warp order. Active
+//                       rows without tokens get zeros.
 // Traffic: dY rows of the tokens of active rows are read once per column chunk (8 KB per token
 // at H = 4096); 16 KB per active row is written.
 #include <atomic>
+#include <mutex>
+
+#include <climits>
 
 #include "sf_common.cuh"
 #include "sf_host.h"
@@ -31,7 +36,8 @@ constexpr int kSumWarps = kSumThreads / 32;
 constexpr int kChunkCols = 256;             // 32 lanes x 8 bf16
 constexpr int kMaxTokens = 16384;
 constexpr int kMaxSlots = 49152;
-constexpr int kMaxSeg = 4096;               // positions a CTA sorts at once in shared memory
+constexpr int kSortThreads = 256;
+constexpr int kSumUnroll = 8;               // token loads in flight per lane
 
 // ws layout: seg_off[slot_cap + 1] int32 | perm[n_tok] int32
 __global__ void __launch_bounds__(kIndexThreads)
@@ -80,12 +86,56 @@ embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int32_t *seg_off, 
     }
 }
 
+// Sorts every active row's segment of positions ascending, in place. Segments hold at most
+// n_tok positions; the host sizes the shared memory for the next power of two above n_tok.
+__global__ void __launch_bounds__(kSortThreads)
+embed_sort_kernel(sf_mask mk, const int32_t *seg_off, int32_t *perm)
+{
+    extern __shared__ int keys[];
+    const int n_act = mk.counts[0];
+    for (int k = blockIdx.x; k < n_act; k += gridDim.x) {
+        const int slot = mk.row_slot[mk.active_rows[k]];
+        if (slot < 0) continue;                       // uniform over the CTA
+        const int b0 = seg_off[slot], n = seg_off[slot + 1] - b0;
+        if (n <= 1) continue;
+        int p2 = 2;
+        while (p2 < n) p2 <<= 1;
+        for (int i = threadIdx.x; i < p2; i += kSortThreads) keys[i] = i < n ? perm[b0 + i] : INT_MAX;
+        __syncthreads();
+        for (int size = 2; size <= p2; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int i = threadIdx.x; i < (p2 >> 1); i += kSortThreads) {
+                    const int lo = 2 * i - (i & (stride - 1));     // pair (lo, lo + stride)
+                    const int hi = lo + stride;
+                    const bool up = (lo & size) == 0;
+                    const int x = keys[lo], y = keys[hi];
+                    if ((x > y) == up) {
+                        keys[lo] = y;
+                        keys[hi] = x;
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        for (int i = threadIdx.x; i < n; i += kSortThreads) perm[b0 + i] = keys[i];
+        __syncthreads();
+    }
+}
+
+__device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 &v)
+{
+    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        acc[2 * e] = __fadd_rn(acc[2 * e], __uint_as_float(ww[e] << 16));
+        acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], __uint_as_float(ww[e] & 0xFFFF0000u));
+    }
+}
+
 __global__ void __launch_bounds__(kSumThreads)
 embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, sf_mask mk, float *G, long long ld_g,
                  const int32_t *seg_off, const int32_t *perm)
 {
-    __shared__ int pos[kMaxSeg];
-    __shared__ int sorted[kMaxSeg];
     __shared__ float part[kSumWarps][kChunkCols];
     const int n_act = mk.counts[0];
     const int nchunks = (H + kChunkCols - 1) / kChunkCols;
@@ -100,47 +150,26 @@ embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, sf_mask mk, float *
         if (slot < 0) continue;
         const int b0 = seg_off[slot], n = seg_off[slot + 1] - b0;
         const int c0 = chunk * kChunkCols + lane * 8;
+        const bool col_ok = c0 < H;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int sb = 0; sb < n; sb += kMaxSeg) {
-            const int m = min(kMaxSeg, n - sb);
-            for (int i = tid; i < m; i += kSumThreads) pos[i] = perm[b0 + sb + i];
-            __syncthreads();
-            // positions are distinct: rank = number of smaller ones
-            for (int i = tid; i < m; i += kSumThreads) {
-                const int p = pos[i];
-                int rank = 0;
-                for (int j = 0; j < m; ++j) rank += pos[j] < p;
-                sorted[rank] = p;
-            }
-            __syncthreads();
-            if (c0 < H) {
-                int i = warp;
-                for (; i + 3 * kSumWarps < m; i += 4 * kSumWarps) {
-                    uint4 v[4];
+        // warp w sums positions w, w + 8, w + 16, ... of the sorted segment, in that order; a
+        // batch holds the warp's next 32 positions, one per lane, handed out by shuffles
+        for (int base = warp; base < n; base += kSumWarps * 32) {
+            const int idx = base + kSumWarps * lane;
+            const int mine = idx < n ? __ldg(perm + b0 + idx) : 0;
+            const int cnt = min(32, (n - base + kSumWarps - 1) / kSumWarps);
+            for (int j0 = 0; j0 < cnt; j0 += kSumUnroll) {
+                uint4 v[kSumUnroll];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        v[u] = __ldg(reinterpret_cast<const uint4 *>(dY + (size_t)sorted[i + u * kSumWarps] * ld_dy + c0));
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint32_t ww[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            acc[2 * e] = __fadd_rn(acc[2 * e], __uint_as_float(ww[e] << 16));
-                            acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], __uint_as_float(ww[e] & 0xFFFF0000u));
-                        }
-                    }
+                for (int u = 0; u < kSumUnroll; ++u) {
+                    const int p = __shfl_sync(0xffffffffu, mine, (j0 + u) & 31);
+                    if (j0 + u < cnt && col_ok)
+                        v[u] = __ldg(reinterpret_cast<const uint4 *>(dY + (size_t)p * ld_dy + c0));
                 }
-                for (; i < m; i += kSumWarps) {
-                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(dY + (size_t)sorted[i] * ld_dy + c0));
-                    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        acc[2 * e] = __fadd_rn(acc[2 * e], __uint_as_float(ww[e] << 16));
-                        acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], __uint_as_float(ww[e] & 0xFFFF0000u));
-                    }
-                }
+                for (int u = 0; u < kSumUnroll; ++u)
+                    if (j0 + u < cnt && col_ok) add_bf16x8(acc, v[u]);
             }
-            __syncthreads();
         }
         // fixed-order combination of the 8 warps' partial sums
 #pragma unroll
@@ -155,6 +184,35 @@ embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, sf_mask mk, float *
         }
         __syncthreads();
     }
+}
+
+// The three launches of one embedding-row gradient, on scratch seg_off[slot_cap + 1] | perm[n_tok].
+int launch_embed(const int32_t *tokens, int n_tok, const void *dY, int H, int64_t ld_dy, const sf_mask &mk,
+                 float *G, int64_t ld_g, int32_t *scratch, uint32_t *dev_status, cudaStream_t st)
+{
+    int32_t *seg_off = scratch;
+    int32_t *perm = seg_off + mk.slot_cap + 1;
+    const size_t smem = (size_t)mk.slot_cap * sizeof(int);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return SF_ERR_CUDA;
+    int p2 = 2;
+    while (p2 < n_tok) p2 <<= 1;
+    const size_t sort_smem = (size_t)p2 * sizeof(int);
+    if (sort_smem > 48 * 1024 &&
+        cudaFuncSetAttribute(embed_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sort_smem) != cudaSuccess)
+        return SF_ERR_CUDA;
+    const int sms = sm_count();
+    if (sms <= 0) return SF_ERR_NO_DEVICE;
+    embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, mk, seg_off, perm, dev_status);
+    if (launch_status() != SF_OK) return SF_ERR_CUDA;
+    embed_sort_kernel<<<sms * 2, kSortThreads, sort_smem, st>>>(mk, seg_off, perm);
+    if (launch_status() != SF_OK) return SF_ERR_CUDA;
+    embed_sum_kernel<<<sms * 4, kSumThreads, 0, st>>>(static_cast<const uint16_t *>(dY), H, ld_dy,
+                                                      mk, G, ld_g, seg_off, perm);
+    return launch_status();
 }
 
 }  // namespace
@@ -181,21 +239,8 @@ extern "C" int sf_embed_grad(const int32_t *tokens, int n_tok, const void *dY, i
     if ((n_tok > 0 && !aligned16(dY)) || !aligned16(G) || !aligned16(ws)) return SF_ERR_ALIGN;
     if (!ws || ws_bytes < sf_embed_grad_ws_bytes(n_tok, mk->slot_cap)) return SF_ERR_ARG;
     if (mk->slot_cap == 0) return SF_OK;
-    cudaStream_t st = as_stream(stream);
-    int32_t *seg_off = static_cast<int32_t *>(ws);
-    int32_t *perm = seg_off + mk->slot_cap + 1;
-    const size_t smem = (size_t)mk->slot_cap * sizeof(int);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return SF_ERR_CUDA;
-    embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, *mk, seg_off, perm, dev_status);
-    if (launch_status() != SF_OK) return SF_ERR_CUDA;
-    const int sms = sm_count();
-    if (sms <= 0) return SF_ERR_NO_DEVICE;
-    embed_sum_kernel<<<sms * 4, kSumThreads, 0, st>>>(static_cast<const uint16_t *>(dY), H, ld_dy,
-                                                      *mk, G, ld_g, seg_off, perm);
-    return launch_status();
+    return launch_embed(tokens, n_tok, dY, H, ld_dy, *mk, G, ld_g, static_cast<int32_t *>(ws), dev_status,
+                        as_stream(stream));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -218,20 +263,54 @@ constexpr int kNoAllocScratchInts = SF_EMBED_NOALLOC_SCRATCH_INTS;
 static __device__ __align__(256) int32_t g_embed_scratch[kNoAllocScratchInts];
 
 constexpr int kMaxDevices = 64;
-std::atomic<int32_t *> g_scratch_addr[kMaxDevices];
 
-// Device address of g_embed_scratch on the current device, looked up once per device (the
-// array's name in host code is only a stand-in for the symbol, not a device pointer).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+// The driver's cuCtxGetCurrent, looked up once through the runtime (the library links no
+// driver library directly).
+CtxGetCurrentFn ctx_get_current()
+{
+    static std::atomic<CtxGetCurrentFn> fn{nullptr};
+    CtxGetCurrentFn f = fn.load(std::memory_order_acquire);
+    if (f) return f;
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+        return nullptr;
+    f = reinterpret_cast<CtxGetCurrentFn>(p);
+    fn.store(f, std::memory_order_release);
+    return f;
+}
+
+struct ScratchAddr {
+    CUcontext ctx;               // the context the address belongs to
+    int32_t *addr;
+};
+ScratchAddr g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mu;
+
+// Device address of g_embed_scratch in the current context (the array's name in host code is
+// only a stand-in for the symbol, not a device pointer). It is looked up with
+// cudaGetSymbolAddress the first time a device is used and again whenever the device's current
+// context is not the one the cached address came from (after cudaDeviceReset, or under another
+// driver-API context), so a stale address is never handed to a kernel.
 int32_t *noalloc_scratch()
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    int32_t *p = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (p) return p;
+    CtxGetCurrentFn get = ctx_get_current();
+    CUcontext ctx = nullptr;
+    if (!get || get(&ctx) != CUDA_SUCCESS) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    ScratchAddr &e = g_scratch_addr[dev];
+    if (ctx && e.addr && e.ctx == ctx) return e.addr;
     void *addr = nullptr;
     if (cudaGetSymbolAddress(&addr, g_embed_scratch) != cudaSuccess || !addr) return nullptr;
-    g_scratch_addr[dev].store(static_cast<int32_t *>(addr), std::memory_order_release);
-    return static_cast<int32_t *>(addr);
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;     // current once the runtime has bound it
+    e.ctx = ctx;
+    e.addr = static_cast<int32_t *>(addr);
+    return e.addr;
 }
 
 }  // namespace
@@ -251,19 +330,5 @@ extern "C" int sf_embed_grad_noalloc(const int32_t *tokens, int n_tok, const voi
     if (mk->slot_cap == 0) return SF_OK;
     int32_t *scratch = noalloc_scratch();
     if (!scratch) return SF_ERR_CUDA;
-    cudaStream_t st = as_stream(stream);
-    int32_t *seg_off = scratch;
-    int32_t *perm = seg_off + mk->slot_cap + 1;
-    const size_t smem = (size_t)mk->slot_cap * sizeof(int);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return SF_ERR_CUDA;
-    embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, *mk, seg_off, perm, dev_status);
-    if (launch_status() != SF_OK) return SF_ERR_CUDA;
-    const int sms = sm_count();
-    if (sms <= 0) return SF_ERR_NO_DEVICE;
-    embed_sum_kernel<<<sms * 4, kSumThreads, 0, st>>>(static_cast<const uint16_t *>(dY), H, ld_dy,
-                                                      *mk, G, ld_g, seg_off, perm);
-    return launch_status();
+    return launch_embed(tokens, n_tok, dY, H, ld_dy, *mk, G, ld_g, scratch, dev_status, as_stream(stream));
 }

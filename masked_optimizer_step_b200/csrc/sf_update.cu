@@ -60,8 +60,10 @@ static_assert(sizeof(UpdBatch) <= 32764, "kernel parameter space");
 // q' = clamp(rint(W / s), -127, 127) with W / s the correctly rounded quotient. The quotient
 // matters only through its rounding to an integer, so it is first formed as W * rcp(s): that
 // product is within 1.6e-5 of W / s and the rounded quotient within 7.6e-6 (|W / s| <= 127.5),
-// so both round to the same integer unless the product lies within 2.3e-5 of a half-integer.
-// Only then (about 1 element in 8,000) is the exact division done.
+// so the two differ by less than 2.3e-5 and can only round differently when the product lies
+// that close to a half-integer. The exact division is taken whenever the product lies within
+// 2^-14 (about 6.1e-5) of a half-integer: a band chosen wider than the 2.3e-5 bound on purpose
+// (about 1 element in 8,000 takes it).
 __device__ __forceinline__ float quant_code(float w, float sp, float rcp, bool fast)
 {
     float qf;

@@ -16,8 +16,6 @@ from tests.gpu_helpers import DEV, bf16_dev, host, i32_dev, mask_host
 
 pytestmark = pytest.mark.gpu
 
-TOL = 2e-3          # the tolerance the embedding-gradient parity tests use
-
 
 def _conductor_mask(V, cap, windows):
     mk = sf.Mask(V, cap, DEV)
@@ -28,9 +26,12 @@ def _conductor_mask(V, cap, windows):
 
 
 def test_noalloc_matches_workspace_version_on_two_calls_in_a_row(sf):
-    V, H, n, cap = 32000, 512, 4096, 4096
+    """Both entry points run the same deterministic kernels on the same inputs, so their outputs
+    must be equal byte for byte. The first call is the larger one (more tokens, more slots), so
+    the second runs over the scratch contents the first left behind."""
+    V, H = 32000, 512
     status = sf.status_word()
-    for call in range(2):
+    for call, (n, cap) in enumerate([(8192, 8192), (2048, 1024)]):
         g = synth.rng(21, "tokens", call)
         windows = [synth.zipf_ids(g, n, V) for _ in range(3)]
         tok = windows[-1]
@@ -46,9 +47,10 @@ def test_noalloc_matches_workspace_version_on_two_calls_in_a_row(sf):
         rows = mh["rows"]
         assert len(rows) > 0
         slots = mh["row_slot"][rows]
-        ref, got = host(G_ref)[slots].astype(np.float64), host(G)[slots].astype(np.float64)
-        floor = 1e-3 * max(np.abs(ref).max(), 1.0)
-        assert np.all(np.abs(got - ref) <= TOL * np.maximum(np.abs(ref), floor)), f"call {call}"
+        assert np.all(slots >= 0)
+        ref, got = host(G_ref)[slots], host(G)[slots]
+        assert got.tobytes() == ref.tobytes(), f"call {call}"
+        assert np.isfinite(got).all()
         # slots no active row holds stay untouched
         unused = np.setdiff1d(np.arange(cap), slots)
         assert np.isnan(host(G)[unused]).all()
