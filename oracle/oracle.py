@@ -58,7 +58,7 @@ def _declare(L):
     L.orc_convert.argtypes = [_I, ctypes.c_long, _P, _P]
     L.orc_window_tokens.restype = _I
     L.orc_window_tokens.argtypes = [_I, _P, _P, _I, _F, _P, _P]
-    L.orc_window_outputs.restype = None
+    L.orc_window_outputs.restype = _I
     L.orc_window_outputs.argtypes = [_I, _P, _P, _I, _F, _P, _P]
     L.orc_mask_lists.restype = None
     L.orc_mask_lists.argtypes = [_I, _P, _P, _P, _P, _P]
@@ -138,14 +138,20 @@ def window_tokens(charge: np.ndarray, tokens, thr: float = 0.01):
 
 def window_outputs(charge: np.ndarray, Y_bf16: np.ndarray, thr: float = 0.01) -> np.ndarray:
     """Fold one window of forward outputs Y[T x R] (bf16 bits) into the charges (in place)."""
+    return window_outputs_counted(charge, Y_bf16, thr)[0]
+
+
+def window_outputs_counted(charge: np.ndarray, Y_bf16: np.ndarray, thr: float = 0.01):
+    """window_outputs, also returning how many outputs were not finite: (words, n_nonfinite).
+    A NaN output is skipped; an infinite one counts as the largest finite bf16 magnitude."""
     R = charge.shape[0]
     Y = _arr(Y_bf16, np.uint16)
     assert Y.ndim == 2 and Y.shape[1] == R
     words = np.zeros(R // 32, dtype=np.uint32)
     h = np.zeros(R, dtype=np.float32)
-    lib().orc_window_outputs(R, _ptr(charge), _ptr(Y), int(Y.shape[0]), float(thr),
-                             _ptr(words), _ptr(h))
-    return words
+    n = lib().orc_window_outputs(R, _ptr(charge), _ptr(Y), int(Y.shape[0]), float(thr),
+                                 _ptr(words), _ptr(h))
+    return words, int(n)
 
 
 def mask_lists(words: np.ndarray):

@@ -146,14 +146,28 @@ int orc_window_tokens(int R, float *charge, const int32_t *tok, int n, float thr
 
 /* Projection row tracker. Y is the forward output, T tokens x R rows, bf16, row-major.
  * Reading of "output magnitudes": a row's magnitude is the largest |Y[t, r]| over the
- * window's tokens, taken on the bf16 values widened to fp32 (exact, independent of order). */
-void orc_window_outputs(int R, float *charge, const uint16_t *Y, int T, float thr,
-                        uint32_t *words, float *h_scratch)
+ * window's tokens, taken on the bf16 values widened to fp32 (exact, independent of order).
+ * Section 2.1 speaks of magnitudes of outputs and says nothing of outputs that are not finite.
+ * Reading for those: a NaN output carries no magnitude and is skipped; an infinite output counts
+ * as the largest finite bfloat16 magnitude (bits 0x7F7F), so the row is as active as a row can
+ * be and every charge stays finite. Returns the number of non-finite outputs seen. */
+int orc_window_outputs(int R, float *charge, const uint16_t *Y, int T, float thr,
+                       uint32_t *words, float *h_scratch)
 {
+    const float largest = orc_bf16_to_f32(0x7F7Fu);
+    int nonfinite = 0;
     for (int r = 0; r < R; ++r) {
         float m = 0.0f;
         for (int t = 0; t < T; ++t) {
             float a = fabsf(orc_bf16_to_f32(Y[(size_t)t * R + r]));
+            if (isnan(a)) {
+                ++nonfinite;
+                continue;
+            }
+            if (isinf(a)) {
+                ++nonfinite;
+                a = largest;
+            }
             if (a > m)
                 m = a;
         }
@@ -164,6 +178,7 @@ void orc_window_outputs(int R, float *charge, const uint16_t *Y, int T, float th
         if (h_scratch[r] > hmax)
             hmax = h_scratch[r];
     orc_charge_fold(R, charge, h_scratch, hmax, thr, words);
+    return nonfinite;
 }
 
 /* The per-step lists every later stage reads: active rows ascending, and the 32-row tiles that

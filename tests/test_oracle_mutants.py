@@ -24,6 +24,10 @@ MUTANTS = {
     "share_wrong_denominator": ("h[r] / hmax;", "h[r] / (hmax + 1.0f);"),
     "tracker_signed_max": ("float a = fabsf(orc_bf16_to_f32(Y[(size_t)t * R + r]));",
                            "float a = orc_bf16_to_f32(Y[(size_t)t * R + r]);"),
+    "tracker_nan_wins": ("            if (isnan(a)) {\n                ++nonfinite;\n                continue;\n            }",
+                         "            if (isnan(a)) {\n                ++nonfinite;\n                a = largest;\n            }"),
+    "tracker_inf_kept": ("                a = largest;\n            }\n            if (a > m)",
+                         "            }\n            if (a > m)"),
     "dw_transposed_operand": ("(double)orc_bf16_to_f32(dX[(size_t)t * R + r])",
                               "(double)orc_bf16_to_f32(dX[(size_t)r * T + t])"),
     "dw_ignores_row_mask": ("continue;                               /* inactive row of an active tile */",

@@ -164,6 +164,32 @@ def test_output_tracker_uses_row_absmax_share():
     assert np.all(charge[4:] < 0.0013)
 
 
+def test_tracker_non_finite_outputs():
+    # A NaN output carries no magnitude; +-inf counts as the largest finite bf16 magnitude
+    # (0x7F7F), so charges stay finite: rows holding an infinity get share 1, the rest share
+    # h / largest in fp32 (subnormal for h = 2 and h = 1). Every non-finite output is counted.
+    T, R = 8, 64
+    g = np.random.default_rng(3)
+    Yb = synth.f32_to_bf16_bits(g.uniform(-0.01, 0.01, size=(T, R)).astype(np.float32))
+    Yb[2, 0] = 0x7F80            # +inf
+    Yb[1, 1] = 0x7FC0            # NaN
+    Yb[5, 1] = 0xC000            # -2.0
+    Yb[4, 2] = 0xFF80            # -inf
+    Yb[:, 3] = 0xFFC1            # NaN (negative sign, other payload) everywhere
+    Yb[0, 4] = 0x3F80            # 1.0
+    charge = np.zeros(R, dtype=np.float32)
+    words, n_bad = orc.window_outputs_counted(charge, Yb)
+    assert n_bad == 3 + T
+    largest = synth.bf16_bits_to_f32(np.array([0x7F7F], np.uint16))[0]
+    assert largest == np.float32(3.3895313892515355e38)
+    half = np.float32(0.5)
+    assert charge[0] == half and charge[2] == half and charge[3] == 0.0
+    assert charge[1] == half * (np.float32(2.0) / largest) and charge[1] > 0
+    assert charge[4] == half * (np.float32(1.0) / largest)
+    assert np.all(np.isfinite(charge))
+    assert words[0] == 0b101 and words[1] == 0
+
+
 def test_tracker_recipe_turns_exactly_the_chosen_rows_on():
     g = synth.rng(2, "tracker", 0)
     R, T = 1024, 512
