@@ -104,7 +104,10 @@ int sf_mask_init(const sf_mask *mk /* host */, sf_stream stream);
  *                      Ids outside [0, R) are ignored and set SF_STATUS_BAD_TOKEN.
  *   SF_SRC_OUTPUT_BF16 ptr = bf16 forward outputs Y [n x ld] (n tokens, columns = rows of W):
  *                      h_r = max over tokens of |Y[t, r]| (the row tracker). ptr and ld*2
- *                      must be 16-byte aligned.
+ *                      must be 16-byte aligned. A NaN output carries no magnitude (it is
+ *                      skipped); an infinite output counts as the largest finite bf16
+ *                      magnitude (3.3895e38), so charges stay finite. Either sets
+ *                      SF_STATUS_NONFINITE.
  *   SF_SRC_HITS_U32    ptr = uint32 hit counts [R] counted by the caller (e.g. on the host).
  *   SF_SRC_WORDS       ptr = uint32 mask words [R/32]: the mask is set directly, the charge
  *                      is not touched (explicit masks).

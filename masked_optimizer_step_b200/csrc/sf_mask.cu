@@ -134,19 +134,41 @@ mask_accum_kernel(const __grid_constant__ MaskBatch b, uint32_t *status)
         m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
         m3 = __vmaxu2(m3, v.w & 0x7FFF7FFFu);
     }
-    const uint32_t mm[4] = {m0, m1, m2, m3};
+    uint32_t mm[4] = {m0, m1, m2, m3};
+    // |bf16| patterns above 0x7F80 are NaN, 0x7F80 is infinity. Reading for non-finite outputs:
+    // a NaN carries no magnitude, an infinity counts as the largest finite bf16 magnitude
+    // (0x7F7F). The packed max is at least 0x7F80 exactly when the segment held one, so only
+    // then is the segment read again with each value mapped first (rare; nothing changes for
+    // finite outputs).
     bool nonfinite = false;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        nonfinite |= (mm[j] & 0xFFFFu) >= 0x7F80u || (mm[j] >> 16) >= 0x7F80u;
+    if (nonfinite) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mm[j] = 0u;
+        for (int tt = t0; tt < t1; ++tt) {
+            const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(Y + (size_t)tt * d.ld + c0));
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t a = w[j] & 0x7FFF7FFFu;
+                a &= ~__vcmpgtu2(a, 0x7F807F80u);          // NaN -> 0
+                a = __vminu2(a, 0x7F7F7F7Fu);              // infinity -> largest finite
+                mm[j] = __vmaxu2(mm[j], a);
+            }
+        }
+        set_status(status, SF_STATUS_NONFINITE);
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const uint32_t half = (mm[j] >> (16 * h)) & 0xFFFFu;
-            nonfinite |= half >= 0x7F80u;
             // widen bf16 magnitude to fp32 bits; non-negative floats order as unsigned ints
             if (half) atomicMax(&d.accum[c0 + 2 * j + h], half << 16);
         }
     }
-    if (nonfinite) set_status(status, SF_STATUS_NONFINITE);
 }
 
 // Finalize, one CTA per mask. Phase 2 runs one warp per 32-row tile (lane = row) and issues the

@@ -94,6 +94,43 @@ def test_tracker_matches_oracle(sf, T, R):
     assert host(status)[0] == 0
 
 
+def test_tracker_non_finite_outputs_match_oracle(sf):
+    """NaN and infinities planted on the host into Y: a NaN carries no magnitude, an infinity
+    counts as the largest finite bf16 magnitude. Charges, words and lists stay bit-exact with the
+    oracle window after window, and SF_STATUS_NONFINITE is set exactly for the windows that held
+    a non-finite output."""
+    R, T, cap = 4096, 1000, 512
+    mk = sf.Mask(R, cap, DEV)
+    sf.sf_mask_init(mk)
+    charge = np.zeros(R, np.float32)
+    nan_patterns = np.array([0x7FC0, 0xFFC0, 0x7F81, 0xFFFF, 0x7FFF], np.uint16)
+    for w, plant in enumerate(["inf+nan", "finite", "nan", "inf+nan"]):
+        g = synth.rng(2, "nonfinite", w)
+        rows = synth.scattered_rows(g, R, 0.01)
+        Y = synth.tracker_outputs(g, T, synth.tracker_gains(R, rows))
+        if "nan" in plant:
+            ts, rs = g.integers(0, T, 300), g.integers(0, R, 300)
+            Y[ts, rs] = nan_patterns[g.integers(0, len(nan_patterns), 300)]
+            Y[:, 77] = 0x7FC0                                  # a row with no magnitude at all
+            Y[: T // 2, rows[0]] = 0xFFC0                      # NaN over half of an active row
+        if "inf" in plant:
+            Y[g.integers(0, T, 5), g.integers(0, R, 5)] = 0x7F80
+            Y[T - 1, 4095] = 0xFF80                            # last token, last column
+            Y[0, 8] = 0x7F80                                   # first token
+        status = sf.status_word()
+        sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_OUTPUT_BF16, bf16_dev(Y), n=T, ld=R)], 0.01, status)
+        words, n_bad = orc.window_outputs_counted(charge, Y)
+        mh = mask_host(mk)
+        assert np.all(np.isfinite(mh["charge"]))
+        assert mh["charge"].tobytes() == charge.tobytes(), plant
+        assert np.array_equal(mh["words"], words), plant
+        r_, t_ = orc.mask_lists(words)
+        assert np.array_equal(mh["rows"], r_) and np.array_equal(mh["tiles"], t_)
+        check_slot_invariants(mh, cap)
+        assert (int(host(status)[0]) & sf.SF_STATUS_NONFINITE != 0) == (n_bad > 0), plant
+        assert (n_bad > 0) == (plant != "finite")
+
+
 def test_many_masks_in_one_call_and_explicit_sources(sf):
     # several masks of different kinds and sizes in one call, each independent
     specs = [(1024, "tokens"), (4096, "output"), (256, "words"), (512, "hits"), (11008, "output")]
