@@ -190,6 +190,21 @@ def masked_dw(dX_bf16: np.ndarray, A_bf16: np.ndarray, words: np.ndarray,
     return out
 
 
+def masked_dw_rows(dX_bf16: np.ndarray, A_bf16: np.ndarray, rows) -> np.ndarray:
+    """dW[r, :] = sum_t dX[t, r] * A[t, :] for the given rows, in fp64, one output row per entry
+    of `rows` (section 2.2's product restricted to chosen rows). The same definition as
+    masked_dw, with the fp64 matrix product of numpy as the summation step: the bf16 inputs
+    widen exactly, so the only difference from the loop is the order of fp64 additions."""
+    dX = _arr(dX_bf16, np.uint16)
+    A = _arr(A_bf16, np.uint16)
+    T, R = dX.shape
+    assert A.shape[0] == T
+    rows = np.asarray(rows, dtype=np.int64)
+    assert rows.ndim == 1 and (rows.size == 0 or (rows.min() >= 0 and rows.max() < R))
+    wide = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return wide(dX[:, rows]).T @ wide(A)
+
+
 def embed_grad(tokens, dY_bf16: np.ndarray, V: int, words: np.ndarray,
                out: np.ndarray | None = None) -> np.ndarray:
     """G[r] = sum of dY rows of the tokens with id r, active rows only (fp64)."""

@@ -190,6 +190,26 @@ def test_tracker_non_finite_outputs():
     assert words[0] == 0b101 and words[1] == 0
 
 
+def test_masked_dw_rows_matches_the_loop():
+    # Integer-valued bf16 inputs keep every fp64 sum exact, so the matrix-product form must equal
+    # the plain loop bit for bit; on N(0,1) inputs they agree to fp64 rounding.
+    g = np.random.default_rng(11)
+    T, R, C = 37, 96, 40
+    dX = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(T, R)).astype(np.float32))
+    A = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(T, C)).astype(np.float32))
+    rows = np.array([0, 5, 31, 32, 64, 95])
+    full = orc.masked_dw(dX, A, synth.words_from_rows(R, rows))
+    got = orc.masked_dw_rows(dX, A, rows)
+    assert got.shape == (len(rows), C)
+    assert np.array_equal(got, full[rows])
+    dX = synth.normal_bf16(g, (T, R))
+    A = synth.normal_bf16(g, (T, C))
+    full = orc.masked_dw(dX, A, synth.words_from_rows(R, rows))
+    np.testing.assert_allclose(orc.masked_dw_rows(dX, A, rows), full[rows], rtol=1e-12, atol=1e-12)
+    # a transposed or shifted operand is caught
+    assert not np.allclose(orc.masked_dw_rows(dX, A, rows[::-1]), full[rows])
+
+
 def test_tracker_recipe_turns_exactly_the_chosen_rows_on():
     g = synth.rng(2, "tracker", 0)
     R, T = 1024, 512
