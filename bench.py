@@ -31,11 +31,11 @@ sys.path.insert(0, ROOT)
 
 METRIC = "sparse step ms & active-row updates/s at 7B shape, 1% active; % of roofline"
 
-# DRAM traffic per layer of each stage (dram__bytes_read.sum + dram__bytes_write.sum), measured
-# with ncu on the 2-layer case of the default workload (scattered masks, 2,048 tokens) and
-# scaled by the layer count; it applies to that workload only.
-TRAFFIC_PER_LAYER = {"masks": (348.541e6 + 3.842e6 + 1.447e6 + 0.000e6) / 2,               # accumulate + finalize
-                     "masked_dw": (173.725e6 + 3.578e6 + 204.643e6 + 8.520e6) / 2}    # gather + main
+# DRAM traffic per launch of a kernel (dram__bytes_read.sum + dram__bytes_write.sum from one ncu
+# capture), keyed by (layers, tokens, masks) of the workload it was captured on; a kernel or
+# workload not listed has none. Entries are removed whenever the kernel changes.
+TRAFFIC_PER_LAUNCH = {}
+TRAFFIC_NOTE = ""
 UNIT = "active-row updates/s"
 SEED = 3
 SWEEP_SEED = 4
@@ -239,7 +239,7 @@ def step_work(model, counts, T):
         upd_bytes += (upd_rows - fresh) * m.C * 24 + fresh * m.C * 20 + upd_rows * 8
         if i >= off:
             track_bytes += T * m.R * 2
-    dw_flops_exec = dw_flops_useful = dw_bytes = 0
+    dw_flops_exec = dw_flops_useful = dw_bytes = gather_bytes = dw_main_bytes = 0
     rows_groups = 0
     for grp in dw_groups(model):
         mats = [model.projs[i].mat for i in grp]
@@ -252,11 +252,17 @@ def step_work(model, counts, T):
         C = mats[0].C
         dw_flops_exec += mt * 128 * C * T * 2
         dw_flops_useful += rows * C * T * 2
-        dw_bytes += T * C * 2 + sum((int(c[0]) - int(c[3])) * C * 4 for c in cs)
-        dw_bytes += T * rows * 2 if rows_mode else sum(int(c[1]) * 32 * T * 2 for c in cs)
+        a_and_rows = T * C * 2 + sum((int(c[0]) - int(c[3])) * C * 4 for c in cs)
+        dx_once = T * rows * 2 if rows_mode else sum(int(c[1]) * 32 * T * 2 for c in cs)
+        dw_bytes += a_and_rows + dx_once
+        # per kernel: the gather reads each active element once and writes it once; the main
+        # kernel streams A once, reads the gathered rows (row mode) or the mask tiles of dX
+        gather_bytes += 2 * T * rows * 2 if rows_mode else 0
+        dw_main_bytes += a_and_rows + dx_once
         rows_groups += rows_mode
     emb = counts[0] if off else None
     return {"dw_flops": dw_flops_exec, "dw_flops_useful": dw_flops_useful, "dw_bytes": dw_bytes,
+            "gather_bytes": gather_bytes, "dw_main_bytes": dw_main_bytes,
             "dw_row_groups": rows_groups, "update_bytes": upd_bytes, "rows_updated": rows_updated,
             "tracker_bytes": track_bytes, "active_rows": int(counts[:, 0].sum()),
             "active_tiles": int(counts[off:, 1].sum()), "emb_rows": int(emb[0]) if emb is not None else 0}
@@ -574,7 +580,7 @@ def _stage_line(model, pipe, hp, status, T, steps, warm, stream, before_step=Non
     names = ("masks", "masked_dw", "embed_grad", "sparse_update")
     st = np.zeros(4)
     for name, e0, e1 in timing:
-        st[names.index(name)] += e0.elapsed_time(e1)
+        st[names.index(name.split(":")[0])] += e0.elapsed_time(e1)
     work = [step_work(model, c, T) for c in log.cpu().numpy()]
     return t0.elapsed_time(t1) / steps, st / steps, work
 
@@ -855,8 +861,11 @@ def main():
     ms_total = t_start.elapsed_time(t_end)
     stage_names = ("masks", "masked_dw", "embed_grad", "sparse_update", "conductor")
     stage_ms = np.zeros(5)
+    pass_ms = {}
     for name, e0, e1 in timing:
-        stage_ms[stage_names.index(name)] += e0.elapsed_time(e1)
+        ms = e0.elapsed_time(e1)
+        stage_ms[stage_names.index(name.split(":")[0])] += ms
+        pass_ms[name] = pass_ms.get(name, 0.0) + ms
     counts = counts_log.cpu().numpy()
     work = [step_work(model, counts[k], T) for k in range(args.steps)]
     rows_updated = sum(w["rows_updated"] for w in work)
@@ -968,33 +977,67 @@ def main():
     stages["step"] = {"hbm_floor_ms": step_bytes / args.steps / (hbm * 1e9) * 1e3,
                       "frac_of_hbm_floor": (step_bytes / (hbm * 1e9)) / (ms_total / 1e3),
                       "algorithmic_gb_per_step": step_bytes / args.steps / 1e9}
-    dominant = max(("masks", "masked_dw", "sparse_update"), key=lambda s: stages[s]["ms_per_step"])
-    d = stages[dominant]
-    traffic = None
-    if args.masks == "scattered" and args.tokens == 2048 and dominant in TRAFFIC_PER_LAYER:
-        traffic = TRAFFIC_PER_LAYER[dominant] * args.layers
-    kernels = {"masks": "sf_mask_update: mask_accum_kernel + mask_finalize_kernel",
-               "masked_dw": "sf_masked_dw: dw_gather_kernel + 3 x masked_dw_kernel",
-               "sparse_update": "sf_sparse_update: update_kernel"}
-    traffic_rate = traffic / (d["ms_per_step"] / 1e3) / 1e9 if traffic else None
+    # ---- per kernel: each pass timed on its own events (the passes are the calls' launches) ----
+    K = args.steps
+    plan0 = plans[0].plans[0]
+    kern = {}
+
+    def hbm_kernel(name, ms_total, bytes_total, launches, what):
+        ms = ms_total / K
+        gbs = bytes_total / (ms_total / 1e3) / 1e9 if ms_total > 0 else 0.0
+        kern[name] = {"ms_per_step": ms, "launches_per_step": launches, "bound": "hbm",
+                      "algorithmic_bytes_per_launch": bytes_total / K / max(launches, 1),
+                      "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, "algorithmic": what}
+
+    n_mask_batches = -(-(plan0.n_masks - (1 if plan0.has_emb else 0)) // sf.SF_MASKS_PER_LAUNCH)
+    if "masks:accum" in pass_ms:
+        hbm_kernel("mask_accum_kernel", pass_ms["masks:accum"], trk_bytes, n_mask_batches,
+                   "tracker pass: Y read once, T*R*2 B per projection")
+        kern["mask_finalize_kernel"] = {"ms_per_step": pass_ms["masks:finalize"] / K,
+                                        "launches_per_step": n_mask_batches, "bound": "latency",
+                                        "note": "one CTA per mask: charges, words, lists, slots"}
+        gather_bytes = sum(w["gather_bytes"] for w in work)
+        main_bytes = sum(w["dw_main_bytes"] for w in work)
+        hbm_kernel("dw_gather_kernel", pass_ms["masked_dw:gather"], gather_bytes, plan0.gather_launches,
+                   "row gather: each active element of dX read once and written once")
+        main_s = pass_ms["masked_dw:main"] / 1e3
+        main_tf = dw_flops / main_s / 1e12 if main_s > 0 else 0.0
+        if dw_flops / (tf_sus * 1e12) >= main_bytes / (hbm * 1e9):
+            kern["masked_dw_kernel"] = {"ms_per_step": main_s * 1e3 / K, "launches_per_step": plan0.dw_launches,
+                                        "bound": "tensor", "algorithmic_flops_per_launch": dw_flops / K / plan0.dw_launches,
+                                        "achieved": main_tf, "peak": tf_sus, "unit": "TFLOP/s", "frac": main_tf / tf_sus,
+                                        "algorithmic": "2*T*C FLOP per executed row (128-row tiles)"}
+        else:
+            hbm_kernel("masked_dw_kernel", pass_ms["masked_dw:main"], main_bytes, plan0.dw_launches,
+                       "A once per group + the gathered rows (row mode) or mask tiles of dX (tile mode) "
+                       "+ dW rows written; the launches are chained, so the span of all of them is timed")
+            kern["masked_dw_kernel"]["tensor_tflops_executed"] = main_tf
+            kern["masked_dw_kernel"]["tensor_frac_executed"] = main_tf / tf_sus
+    hbm_kernel("update_kernel", stage_ms[3], upd_bytes, -(-len(plan0.upd_arr) // sf.SF_MATS_PER_LAUNCH),
+               "24 B per active element (20 on fresh rows) + 8 B per row")
+    if stage_ms[2] > 0:
+        kern["embed (index + sort + sum)"] = {"ms_per_step": stage_ms[2] / K, "launches_per_step": 3,
+                                              "stream": "side (overlapped)" if not args.no_overlap_embedding else "main"}
+    rated = [k for k, v in kern.items() if v.get("bound") in ("hbm", "tensor")]
+    dominant = max(rated, key=lambda k: kern[k]["ms_per_step"])
+    d = kern[dominant]
+    workload_key = (args.layers, args.tokens, args.masks)
+    traffic = TRAFFIC_PER_LAUNCH.get(dominant, {}).get(workload_key)
     roofline = {"bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-                "frac": d["frac"], "traffic": traffic, "traffic_unit": "bytes per step (one call)",
-                "traffic_gbs": traffic_rate,
-                "traffic_frac": traffic_rate / hbm if traffic_rate else None,
-                "traffic_note": "DRAM bytes the call actually moves (ncu) over its event-timed duration: the "
-                                "row gather reads dX at DRAM granularity (~128 B per 64-column window "
-                                "holding an active row), so traffic exceeds the 2 B per gathered element "
-                                "counted in the algorithmic bytes" if d["bound"] == "hbm" and dominant == "masked_dw"
-                                else None,
-                "kernel": kernels[dominant], "peak_source": peak_src,
+                "frac": d["frac"], "traffic": traffic,
+                "traffic_unit": "DRAM bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                "traffic_note": TRAFFIC_NOTE if traffic is not None else
+                                "no ncu capture of this kernel on this workload with the current build",
+                "kernel": dominant, "launches_per_step": d["launches_per_step"],
+                "ms_per_launch": d["ms_per_step"] / max(d["launches_per_step"], 1),
+                "peak_source": peak_src,
                 "peak_kind": "sustained bf16 (kernel timed inside a long step)" if d["bound"] == "tensor" else "hbm copy",
                 "algorithmic": d["algorithmic"]}
-
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32", "data": "synthetic",
-        "config": workload_config(args), "roofline": roofline, "stages": stages,
+        "config": workload_config(args), "roofline": roofline, "kernels": kern, "stages": stages,
         "gpu_launches": plans[0].launches() * args.steps,
         "clocks": clk,
         "per_step": {"active_rows": work[-1]["active_rows"], "rows_updated": work[-1]["rows_updated"],

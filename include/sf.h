@@ -300,6 +300,28 @@ int sf_checkpoint_save(const sf_matrix *mats /* host [n] */, const sf_checkpoint
 int sf_checkpoint_restore(const sf_matrix *mats /* host [n] */, const sf_checkpoint *ck /* host [n] */,
                           int n, uint32_t *dev_status, sf_stream stream);
 
+/* ---- sf_mask_update_phase / sf_masked_dw_phase: one pass of a two-pass call ------------------
+ * No counterpart in the paper: a measurement aid. sf_mask_update and sf_masked_dw each run two
+ * passes; these variants enqueue only the pass `phase` names, so that a caller can record CUDA
+ * events between the passes and time each kernel on its own. SF_PHASE_FIRST then SF_PHASE_SECOND
+ * on one stream, with the same arguments and nothing in between that touches their buffers,
+ * does exactly what the full call (SF_PHASE_ALL) does.
+ *   sf_mask_update: FIRST = the activity pass (token histogram / column absmax into accum);
+ *                   SECOND = the finalize pass (charges, mask words, lists, slots).
+ *   sf_masked_dw:   FIRST = the row gather of the groups that run in row mode (nothing when
+ *                   ws is NULL); SECOND = the main tensor-core launches.
+ * Errors: those of the full call, and SF_ERR_ARG for an unknown phase.
+ */
+#define SF_PHASE_ALL    0
+#define SF_PHASE_FIRST  1
+#define SF_PHASE_SECOND 2
+
+int sf_mask_update_phase(const sf_mask *masks /* host [n_masks] */,
+                         const sf_mask_src *srcs /* host [n_masks] */, int n_masks, float threshold,
+                         int phase, uint32_t *dev_status, sf_stream stream);
+int sf_masked_dw_phase(const sf_dw_problem *probs /* host [n] */, int n, void *ws, size_t ws_bytes,
+                       int phase, uint32_t *dev_status, sf_stream stream);
+
 /* ---- helpers (not on the hot path) ------------------------------------------------------ */
 
 /* Quantise a full-precision matrix into the int8 + scale + residual storage of section 2.3

@@ -28,6 +28,10 @@ SF_SRC_OUTPUT_BF16 = 1
 SF_SRC_HITS_U32 = 2
 SF_SRC_WORDS = 3
 
+SF_PHASE_ALL = 0
+SF_PHASE_FIRST = 1
+SF_PHASE_SECOND = 2
+
 SF_DW_MAX_PER_LAUNCH = 96
 SF_MASKS_PER_LAUNCH = 240
 SF_MATS_PER_LAUNCH = 256
@@ -89,6 +93,10 @@ def load():
     L.sf_mask_update.argtypes = [ctypes.POINTER(sf_mask), ctypes.POINTER(sf_mask_src), ctypes.c_int,
                                  _F, _P, _P]
     L.sf_masked_dw.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int, _P, ctypes.c_size_t, _P, _P]
+    L.sf_mask_update_phase.argtypes = [ctypes.POINTER(sf_mask), ctypes.POINTER(sf_mask_src), ctypes.c_int,
+                                       _F, ctypes.c_int, _P, _P]
+    L.sf_masked_dw_phase.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int, _P, ctypes.c_size_t,
+                                     ctypes.c_int, _P, _P]
     L.sf_masked_dw_ws_bytes.restype = ctypes.c_size_t
     L.sf_masked_dw_ws_bytes.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int]
     L.sf_embed_grad_ws_bytes.restype = ctypes.c_size_t
@@ -106,7 +114,7 @@ def load():
         getattr(L, name).argtypes = [ctypes.POINTER(sf_matrix), ctypes.POINTER(sf_checkpoint), ctypes.c_int, _P, _P]
         getattr(L, name).restype = ctypes.c_int
     for name in ("sf_mask_init", "sf_mask_update", "sf_masked_dw", "sf_embed_grad", "sf_adam_tables",
-                 "sf_sparse_update", "sf_quantize_init"):
+                 "sf_sparse_update", "sf_quantize_init", "sf_mask_update_phase", "sf_masked_dw_phase"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -219,6 +227,15 @@ def sf_mask_update(masks, srcs, threshold: float = 0.01, status=None, stream=Non
            "sf_mask_update")
 
 
+def sf_mask_update_phase(masks, srcs, phase: int, threshold: float = 0.01, status=None, stream=None):
+    """One pass of sf_mask_update (SF_PHASE_FIRST: activity, SF_PHASE_SECOND: finalize)."""
+    n = len(masks)
+    arr_m = (sf_mask * n)(*[m.struct() for m in masks])
+    arr_s = (sf_mask_src * n)(*[s.c for s in srcs])
+    _check(load().sf_mask_update_phase(arr_m, arr_s, n, threshold, phase, _ptr(status), _stream(stream)),
+           "sf_mask_update_phase")
+
+
 def dw_problem(dX, A, mask: Mask, dW) -> Desc:
     """dX [T x R] bf16, A [T x C] bf16, dW [slot_cap x C] fp32 (row = slot)."""
     T, R = dX.shape
@@ -247,6 +264,15 @@ def sf_masked_dw(problems, status=None, stream=None, ws=None):
     arr = (sf_dw_problem * n)(*[p.c for p in problems])
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(load().sf_masked_dw(arr, n, _ptr(ws), nbytes, _ptr(status), _stream(stream)), "sf_masked_dw")
+
+
+def sf_masked_dw_phase(problems, phase: int, status=None, stream=None, ws=None):
+    """One pass of sf_masked_dw (SF_PHASE_FIRST: row gather, SF_PHASE_SECOND: main launches)."""
+    n = len(problems)
+    arr = (sf_dw_problem * n)(*[p.c for p in problems])
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(load().sf_masked_dw_phase(arr, n, _ptr(ws), nbytes, phase, _ptr(status), _stream(stream)),
+           "sf_masked_dw_phase")
 
 
 def sf_embed_grad_ws_bytes(n_tok: int, slot_cap: int) -> int:

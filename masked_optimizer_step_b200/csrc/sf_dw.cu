@@ -609,9 +609,10 @@ extern "C" size_t sf_masked_dw_ws_bytes(const sf_dw_problem *probs, int n)
     return total;
 }
 
-extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t ws_bytes,
-                            uint32_t *dev_status, sf_stream stream)
+extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, size_t ws_bytes, int phase,
+                                  uint32_t *dev_status, sf_stream stream)
 {
+    if (phase != SF_PHASE_ALL && phase != SF_PHASE_FIRST && phase != SF_PHASE_SECOND) return SF_ERR_ARG;
     if (n < 0 || (n > 0 && !probs)) return SF_ERR_ARG;
     for (int i = 0; i < n; ++i) {
         const sf_dw_problem &p = probs[i];
@@ -648,7 +649,7 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
     auto row_ok = [&](const HostGroup &hg) { return use_ws && probs[hg.first].T > 0 && hg.mcap > 0; };
 
     // ---- gather pass: every group of the call, in as few launches as the parameters allow ----
-    GatherBatch *gb = (rc == SF_OK && use_ws) ? new GatherBatch : nullptr;
+    GatherBatch *gb = (rc == SF_OK && use_ws && phase != SF_PHASE_SECOND) ? new GatherBatch : nullptr;
     for (int gi = 0; gb && rc == SF_OK && gi < ng;) {
         memset(gb, 0, sizeof(*gb));
         int tok_blocks = 1;
@@ -687,10 +688,10 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
     size_t all = 0;
     for (int k = 0; k < ng; ++k) all += launch_bytes(groups[k]);
     int n_launch = (int)((all + payload - 1) / payload);
-    DwBatch *batch = rc == SF_OK ? new DwBatch : nullptr;
+    DwBatch *batch = (rc == SF_OK && phase != SF_PHASE_FIRST) ? new DwBatch : nullptr;
     int gi = 0;
     int n_main_launches = 0;
-    for (int li = 0; rc == SF_OK && gi < ng; ++li) {
+    for (int li = 0; batch && rc == SF_OK && gi < ng; ++li) {
         size_t left = 0;
         for (int k = gi; k < ng; ++k) left += launch_bytes(groups[k]);
         const int launches_left = n_launch - li > 1 ? n_launch - li : 1;
@@ -779,4 +780,10 @@ extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t 
     delete batch;
     delete[] groups;
     return rc;
+}
+
+extern "C" int sf_masked_dw(const sf_dw_problem *probs, int n, void *ws, size_t ws_bytes,
+                            uint32_t *dev_status, sf_stream stream)
+{
+    return sf_masked_dw_phase(probs, n, ws, ws_bytes, SF_PHASE_ALL, dev_status, stream);
 }

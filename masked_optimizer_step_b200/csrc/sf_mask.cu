@@ -387,9 +387,10 @@ extern "C" int sf_mask_init(const sf_mask *mk, sf_stream stream)
     return launch_status();
 }
 
-extern "C" int sf_mask_update(const sf_mask *masks, const sf_mask_src *srcs, int n_masks,
-                              float threshold, uint32_t *dev_status, sf_stream stream)
+extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *srcs, int n_masks,
+                                    float threshold, int phase, uint32_t *dev_status, sf_stream stream)
 {
+    if (phase != SF_PHASE_ALL && phase != SF_PHASE_FIRST && phase != SF_PHASE_SECOND) return SF_ERR_ARG;
     if (n_masks < 0 || (n_masks > 0 && (!masks || !srcs))) return SF_ERR_ARG;
     if (!(threshold >= 0.0f)) return SF_ERR_ARG;
     // validate everything before the first launch
@@ -476,12 +477,20 @@ extern "C" int sf_mask_update(const sf_mask *masks, const sf_mask_src *srcs, int
                 ctas += d.col_blocks * d.tok_segs;
         }
         batch.total_ctas = ctas;
-        if (ctas > 0) {
+        if (ctas > 0 && phase != SF_PHASE_SECOND) {
             mask_accum_kernel<<<ctas, kAccumThreads, 0, st>>>(batch, dev_status);
             if (launch_status() != SF_OK) return SF_ERR_CUDA;
         }
-        mask_finalize_kernel<<<cnt, kFinalizeThreads, fin_smem, st>>>(batch, threshold, dev_status);
-        if (launch_status() != SF_OK) return SF_ERR_CUDA;
+        if (phase != SF_PHASE_FIRST) {
+            mask_finalize_kernel<<<cnt, kFinalizeThreads, fin_smem, st>>>(batch, threshold, dev_status);
+            if (launch_status() != SF_OK) return SF_ERR_CUDA;
+        }
     }
     return SF_OK;
+}
+
+extern "C" int sf_mask_update(const sf_mask *masks, const sf_mask_src *srcs, int n_masks,
+                              float threshold, uint32_t *dev_status, sf_stream stream)
+{
+    return sf_mask_update_phase(masks, srcs, n_masks, threshold, SF_PHASE_ALL, dev_status, stream);
 }

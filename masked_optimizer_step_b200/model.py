@@ -237,24 +237,24 @@ class StepPlan:
         sf._check(self.lib.sf_mask_update(self.mask_arr, self.src_arr, 1, self.threshold, status, stream),
                   "sf_mask_update")
 
-    def masks_projections(self, status, stream):
-        """The row trackers of every projection of the plan, as one call."""
+    def masks_projections(self, status, stream, phase: int = sf.SF_PHASE_ALL):
+        """The row trackers of every projection of the plan, as one call (or one of its passes)."""
         off = 1 if self.has_emb else 0
         n = self.n_masks - off
         if n <= 0:
             return
-        sf._check(self.lib.sf_mask_update(self.proj_mask_arr, self.proj_src_arr, n, self.threshold, status,
-                                          stream), "sf_mask_update")
+        sf._check(self.lib.sf_mask_update_phase(self.proj_mask_arr, self.proj_src_arr, n, self.threshold, phase,
+                                                status, stream), "sf_mask_update")
 
     def masks(self, status, stream):
         sf._check(self.lib.sf_mask_update(self.mask_arr, self.src_arr, self.n_masks, self.threshold,
                                           status, stream), "sf_mask_update")
 
-    def dw(self, status, stream):
+    def dw(self, status, stream, phase: int = sf.SF_PHASE_ALL):
         if self.n_dw == 0:
             return
-        sf._check(self.lib.sf_masked_dw(self.dw_arr, self.n_dw, self.dw_ws.data_ptr(), self.dw_ws.numel(),
-                                        status, stream), "sf_masked_dw")
+        sf._check(self.lib.sf_masked_dw_phase(self.dw_arr, self.n_dw, self.dw_ws.data_ptr(), self.dw_ws.numel(),
+                                              phase, status, stream), "sf_masked_dw")
 
     def embed(self, status, stream):
         if not self.has_emb:
@@ -336,7 +336,10 @@ class Pipeline:
 
     def step(self, hp: sf.AdamParams, status, main, timing: list | None = None):
         """Issue one step. main: the torch stream the step belongs to; timing: if a list, gets
-        (stage, start event, end event) for every call (events on the call's own stream)."""
+        (stage, start event, end event) for every call (events on the call's own stream). With the
+        embedding on the side stream, the masks and dW calls are then issued pass by pass, each
+        pass on its own events ("masks:accum", "masks:finalize", "masked_dw:gather",
+        "masked_dw:main"); the passes are the same launches the full calls make."""
         side = self.side
         sp_main, sp_side = main.cuda_stream, side.cuda_stream
 
@@ -357,8 +360,14 @@ class Pipeline:
             timed("conductor", side, lambda: plan.masks_embedding(status, sp_side))
             timed("embed_grad", side, lambda: plan.embed(status, sp_side))
             self.emb_done.record(side)
-            timed("masks", main, lambda: plan.masks_projections(status, sp_main))
-            timed("masked_dw", main, lambda: plan.dw(status, sp_main))
+            if timing is None:
+                plan.masks_projections(status, sp_main)
+                plan.dw(status, sp_main)
+            else:                                    # each pass of the two-pass calls on its own events
+                timed("masks:accum", main, lambda: plan.masks_projections(status, sp_main, sf.SF_PHASE_FIRST))
+                timed("masks:finalize", main, lambda: plan.masks_projections(status, sp_main, sf.SF_PHASE_SECOND))
+                timed("masked_dw:gather", main, lambda: plan.dw(status, sp_main, sf.SF_PHASE_FIRST))
+                timed("masked_dw:main", main, lambda: plan.dw(status, sp_main, sf.SF_PHASE_SECOND))
             main.wait_event(self.emb_done)
             timed("sparse_update", main, lambda: plan.update(hp, status, sp_main))
             return

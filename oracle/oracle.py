@@ -60,6 +60,10 @@ def _declare(L):
     L.orc_window_tokens.argtypes = [_I, _P, _P, _I, _F, _P, _P]
     L.orc_window_outputs.restype = _I
     L.orc_window_outputs.argtypes = [_I, _P, _P, _I, _F, _P, _P]
+    L.orc_window_activity.restype = None
+    L.orc_window_activity.argtypes = [_I, _P, _P, _F, _P]
+    L.orc_row_magnitudes.restype = _I
+    L.orc_row_magnitudes.argtypes = [_I, _P, _I, _P]
     L.orc_mask_lists.restype = None
     L.orc_mask_lists.argtypes = [_I, _P, _P, _P, _P, _P]
     L.orc_moments_follow_mask.restype = None
@@ -152,6 +156,25 @@ def window_outputs_counted(charge: np.ndarray, Y_bf16: np.ndarray, thr: float = 
     n = lib().orc_window_outputs(R, _ptr(charge), _ptr(Y), int(Y.shape[0]), float(thr),
                                  _ptr(words), _ptr(h))
     return words, int(n)
+
+
+def window_activity(charge: np.ndarray, h: np.ndarray, thr: float = 0.01) -> np.ndarray:
+    """The charge rule applied to activities h[R] given directly (in place on charge)."""
+    R = charge.shape[0]
+    h = _arr(np.asarray(h, dtype=np.float32), np.float32)
+    assert h.shape == (R,)
+    words = np.zeros(R // 32, dtype=np.uint32)
+    lib().orc_window_activity(R, _ptr(charge), _ptr(h), float(thr), _ptr(words))
+    return words
+
+
+def row_magnitudes(Y_bf16: np.ndarray):
+    """The tracker's activities: (h[R] = largest |Y[t, r]| over tokens, non-finite count)."""
+    Y = _arr(Y_bf16, np.uint16)
+    T, R = Y.shape
+    h = np.zeros(R, dtype=np.float32)
+    n = lib().orc_row_magnitudes(R, _ptr(Y), T, _ptr(h))
+    return h, int(n)
 
 
 def mask_lists(words: np.ndarray):

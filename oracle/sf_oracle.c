@@ -181,6 +181,45 @@ int orc_window_outputs(int R, float *charge, const uint16_t *Y, int T, float thr
     return nonfinite;
 }
 
+/* The charge rule of one window from the rows' activities h[R] given directly (the busiest row
+ * is found here). window_tokens and window_outputs are this rule applied to the activities they
+ * count; split across several processes, each counts its share of the window's tokens and the
+ * shares are combined (summed hit counts, largest magnitude) before the rule is applied once. */
+void orc_window_activity(int R, float *charge, const float *h, float thr, uint32_t *words)
+{
+    float hmax = 0.0f;
+    for (int r = 0; r < R; ++r)
+        if (h[r] > hmax)
+            hmax = h[r];
+    orc_charge_fold(R, charge, h, hmax, thr, words);
+}
+
+/* The row tracker's activities alone: h[r] = largest |Y[t, r]| over the T tokens, with the
+ * reading for non-finite outputs of orc_window_outputs. Returns the number of non-finite outputs. */
+int orc_row_magnitudes(int R, const uint16_t *Y, int T, float *h)
+{
+    const float largest = orc_bf16_to_f32(0x7F7Fu);
+    int nonfinite = 0;
+    for (int r = 0; r < R; ++r) {
+        float m = 0.0f;
+        for (int t = 0; t < T; ++t) {
+            float a = fabsf(orc_bf16_to_f32(Y[(size_t)t * R + r]));
+            if (isnan(a)) {
+                ++nonfinite;
+                continue;
+            }
+            if (isinf(a)) {
+                ++nonfinite;
+                a = largest;
+            }
+            if (a > m)
+                m = a;
+        }
+        h[r] = m;
+    }
+    return nonfinite;
+}
+
 /* The per-step lists every later stage reads: active rows ascending, and the 32-row tiles that
  * hold at least one active row, ascending. Returns nothing; counts go to n_rows / n_tiles. */
 void orc_mask_lists(int R, const uint32_t *words, int32_t *rows, int32_t *n_rows,

@@ -37,8 +37,9 @@ def _bits(t):
 
 
 def _dw_row_errors(got, ref):
-    """Per-row relative error with a floor of 1e-3 of the row's largest entry."""
-    floor = 1e-3 * np.maximum(np.abs(ref).max(axis=1, keepdims=True), 1e-30)
+    """Per-row largest relative error |got - ref| / max(|ref|, floor), the floor being 1e-3 of the
+    largest |entry| of the projection's checked dW (the dW tolerance's definition)."""
+    floor = 1e-3 * max(float(np.abs(ref).max()), 1e-30)
     return np.max(np.abs(got.astype(np.float64) - ref) / np.maximum(np.abs(ref), floor), axis=1)
 
 

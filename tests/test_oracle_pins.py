@@ -210,6 +210,31 @@ def test_masked_dw_rows_matches_the_loop():
     assert not np.allclose(orc.masked_dw_rows(dX, A, rows[::-1]), full[rows])
 
 
+def test_activity_rule_split_over_token_shares():
+    # The rule applied to combined activities equals the windows counted in one piece: hit
+    # counts add over disjoint token shares, row magnitudes combine by max (and so does the
+    # non-finite handling), for any split of the tokens.
+    g = np.random.default_rng(5)
+    R, V, T = 256, 256, 96
+    tok = synth.zipf_ids(g, T, V)
+    c1, c2 = np.zeros(V, np.float32), np.zeros(V, np.float32)
+    w1, _ = orc.window_tokens(c1, tok)
+    hits = np.bincount(tok[:40], minlength=V) + np.bincount(tok[40:], minlength=V)
+    w2 = orc.window_activity(c2, hits.astype(np.float32))
+    assert c1.tobytes() == c2.tobytes() and np.array_equal(w1, w2)
+    Y = synth.tracker_outputs(g, T, synth.tracker_gains(R, synth.scattered_rows(g, R, 0.03)))
+    Y[5, 7], Y[60, 9] = 0x7F80, 0x7FC0
+    c1, c2 = np.zeros(R, np.float32), np.zeros(R, np.float32)
+    w1, n1 = orc.window_outputs_counted(c1, Y)
+    (ha, na), (hb, nb) = orc.row_magnitudes(Y[:33]), orc.row_magnitudes(Y[33:])
+    w2 = orc.window_activity(c2, np.maximum(ha, hb))
+    assert c1.tobytes() == c2.tobytes() and np.array_equal(w1, w2) and n1 == na + nb == 2
+    # an empty window is pure decay
+    c3 = c1.copy()
+    orc.window_activity(c3, np.zeros(R, np.float32))
+    assert c3.tobytes() == (np.float32(0.5) * c1).tobytes()
+
+
 def test_tracker_recipe_turns_exactly_the_chosen_rows_on():
     g = synth.rng(2, "tracker", 0)
     R, T = 1024, 512
