@@ -6,13 +6,11 @@
 // upstream gradients dY[t] over the batch positions t holding token r, and only rows the
 // conductor marks active are computed and stored.
 //
-// Three launches:
+// Two launches:
 //   embed_index_kernel  one CTA: for every token whose row is active, its slot; per-slot counts
 //                       (shared-memory atomics, exact), an exclusive scan into segment offsets,
-//                       and a scatter of token positions into their slot's segment of ws.
-//   embed_sort_kernel   one CTA per active row at a time: the row's segment is sorted ascending
-//                       in shared memory (bitonic network), once per row, so the sum order
-//                       never depends on the order the scatter's atomics happened to take.
+//                       and a stable scatter of token positions into their slot's segment of ws
+//                       (ascending within a segment, so the sum order is fixed).
 //   embed_sum_kernel    persistent: one item = (active row, 256-column chunk). 8 warps each
 //                       sum every 8th token of the row's sorted segment with 16-byte loads (eight
 //                       in flight per lane) and the partial sums are added in warp order. Active
@@ -36,7 +34,6 @@ constexpr int kSumWarps = kSumThreads / 32;
 constexpr int kChunkCols = 256;             // 32 lanes x 8 bf16
 constexpr int kMaxTokens = 16384;
 constexpr int kMaxSlots = 49152;
-constexpr int kSortThreads = 256;
 constexpr int kSumUnroll = 8;               // token loads in flight per lane
 
 // ws layout: seg_off[slot_cap + 1] int32 | perm[n_tok] int32
@@ -78,47 +75,31 @@ embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int32_t *seg_off, 
     }
     if (threadIdx.x == 0) seg_off[cap] = s_run;
     __syncthreads();
-    for (int t = threadIdx.x; t < n_tok; t += blockDim.x) {
-        const int r = tok[t];
-        if (r < 0 || r >= mk.R || !((mk.words[r >> 5] >> (r & 31)) & 1u)) continue;
-        const int s = mk.row_slot[r];
-        if (s >= 0) perm[seg_off[s] + atomicAdd(&cnt[s], 1)] = t;
-    }
-}
-
-// Sorts every active row's segment of positions ascending, in place. Segments hold at most
-// n_tok positions; the host sizes the shared memory for the next power of two above n_tok.
-__global__ void __launch_bounds__(kSortThreads)
-embed_sort_kernel(sf_mask mk, const int32_t *seg_off, int32_t *perm)
-{
-    extern __shared__ int keys[];
-    const int n_act = mk.counts[0];
-    for (int k = blockIdx.x; k < n_act; k += gridDim.x) {
-        const int slot = mk.row_slot[mk.active_rows[k]];
-        if (slot < 0) continue;                       // uniform over the CTA
-        const int b0 = seg_off[slot], n = seg_off[slot + 1] - b0;
-        if (n <= 1) continue;
-        int p2 = 2;
-        while (p2 < n) p2 <<= 1;
-        for (int i = threadIdx.x; i < p2; i += kSortThreads) keys[i] = i < n ? perm[b0 + i] : INT_MAX;
-        __syncthreads();
-        for (int size = 2; size <= p2; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                for (int i = threadIdx.x; i < (p2 >> 1); i += kSortThreads) {
-                    const int lo = 2 * i - (i & (stride - 1));     // pair (lo, lo + stride)
-                    const int hi = lo + stride;
-                    const bool up = (lo & size) == 0;
-                    const int x = keys[lo], y = keys[hi];
-                    if ((x > y) == up) {
-                        keys[lo] = y;
-                        keys[hi] = x;
-                    }
-                }
-                __syncthreads();
-            }
+    // Stable scatter: a slot's positions land in ascending order. Tokens go in rounds of
+    // blockDim (one per thread, in order); inside a warp, lanes holding the same slot rank
+    // themselves by lane; across warps, each warp's group leaders claim their slots' next places
+    // in warp order, one warp per barrier step. So the sum order below never depends on timing.
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int base = 0; base < n_tok; base += blockDim.x) {
+        const int t = base + threadIdx.x;
+        int s = -1;
+        if (t < n_tok) {
+            const int r = tok[t];
+            if (r >= 0 && r < mk.R && ((mk.words[r >> 5] >> (r & 31)) & 1u)) s = mk.row_slot[r];
         }
-        for (int i = threadIdx.x; i < n; i += kSortThreads) perm[b0 + i] = keys[i];
-        __syncthreads();
+        const uint32_t peers = __match_any_sync(0xffffffffu, s);
+        const int leader = __ffs(peers) - 1;
+        int place = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            if (warp == w && s >= 0 && lane == leader) {
+                place = cnt[s];
+                cnt[s] = place + __popc(peers);
+            }
+            __syncthreads();
+        }
+        place = __shfl_sync(0xffffffffu, place, leader);
+        if (s >= 0) perm[seg_off[s] + place + __popc(peers & lt)] = t;
     }
 }
 
@@ -186,7 +167,7 @@ embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, sf_mask mk, float *
     }
 }
 
-// The three launches of one embedding-row gradient, on scratch seg_off[slot_cap + 1] | perm[n_tok].
+// The two launches of one embedding-row gradient, on scratch seg_off[slot_cap + 1] | perm[n_tok].
 int launch_embed(const int32_t *tokens, int n_tok, const void *dY, int H, int64_t ld_dy, const sf_mask &mk,
                  float *G, int64_t ld_g, int32_t *scratch, uint32_t *dev_status, cudaStream_t st)
 {
@@ -197,18 +178,9 @@ int launch_embed(const int32_t *tokens, int n_tok, const void *dY, int H, int64_
         cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return SF_ERR_CUDA;
-    int p2 = 2;
-    while (p2 < n_tok) p2 <<= 1;
-    const size_t sort_smem = (size_t)p2 * sizeof(int);
-    if (sort_smem > 48 * 1024 &&
-        cudaFuncSetAttribute(embed_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sort_smem) != cudaSuccess)
-        return SF_ERR_CUDA;
     const int sms = sm_count();
     if (sms <= 0) return SF_ERR_NO_DEVICE;
     embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, mk, seg_off, perm, dev_status);
-    if (launch_status() != SF_OK) return SF_ERR_CUDA;
-    embed_sort_kernel<<<sms * 2, kSortThreads, sort_smem, st>>>(mk, seg_off, perm);
     if (launch_status() != SF_OK) return SF_ERR_CUDA;
     embed_sum_kernel<<<sms * 4, kSumThreads, 0, st>>>(static_cast<const uint16_t *>(dY), H, ld_dy,
                                                       mk, G, ld_g, seg_off, perm);

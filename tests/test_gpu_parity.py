@@ -105,7 +105,7 @@ def test_tracker_non_finite_outputs_match_oracle(sf):
     charge = np.zeros(R, np.float32)
     nan_patterns = np.array([0x7FC0, 0xFFC0, 0x7F81, 0xFFFF, 0x7FFF], np.uint16)
     for w, plant in enumerate(["inf+nan", "finite", "nan", "inf+nan"]):
-        g = synth.rng(2, "nonfinite", w)
+        g = synth.rng(2, "misc", 31, w)
         rows = synth.scattered_rows(g, R, 0.01)
         Y = synth.tracker_outputs(g, T, synth.tracker_gains(R, rows))
         if "nan" in plant:
