@@ -22,14 +22,17 @@
 //              scattered (at 1% scattered rows, a live tile holds ~1.2 active rows).
 // Row mode is used when the group's active rows fit the scratch and it needs fewer M-tiles.
 //
-// CTA (1 per SM, 192 threads, warp-specialised, persistent over the units of the launch):
+// CTA (1 per SM, 320 threads, warp-specialised, persistent over the units of the launch):
 //   warp 0      TMA producer: per 64-token stage, four 32-row boxes of the A-operand
 //               (SWIZZLE_64B) and four 64-column boxes of A (SWIZZLE_128B) into a 4-deep ring;
 //   warp 1      allocates 512 TMEM columns, one thread issues tcgen05.mma kind::f16
-//               (M=128, N=256, K=16, bf16 in, fp32 accumulate) into one of two 256-column
-//               accumulators and commits stage releases / accumulator-ready to mbarriers;
-//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns at a time (warp w reads TMEM lanes
-//               32*(w%4)..), maps each lane to its weight row and slot, stores fp32 rows of dW.
+//               (M=128, N=256, K=16, bf16 in, fp32 accumulate). Each chunk of 1024 tokens goes
+//               into one of two 256-column TMEM buffers, starting from zero; the thread commits
+//               stage releases and chunk-ready signals to mbarriers;
+//   warps 2-9   epilogue: two warps per TMEM lane quarter (warp w reads lanes 32*(w%4)..), one
+//               per 128-column half; each adds every finished chunk into fp32 registers
+//               (round to nearest), then maps each lane to its weight row and slot and stores
+//               the row of dW once per unit.
 // Every mbarrier wait is bounded (2 s): on expiry the CTA raises SF_STATUS_WAIT_TIMEOUT, drains
 // its own TMA loads, frees its TMEM and exits.
 #include <stdlib.h>
@@ -42,13 +45,7 @@ namespace sf {
 namespace {
 
 constexpr int BM = 128;                 // rows per unit
-#ifndef SF_DW_BN
-#define SF_DW_BN 256
-#endif
-constexpr int BN = SF_DW_BN;            // columns per unit
-constexpr int MMA_N = BN > 256 ? 256 : BN;   // N of one tcgen05.mma (at most 256)
-constexpr int NSUB = BN / MMA_N;             // MMAs per 16-token step across the unit's columns
-static_assert(BN % MMA_N == 0 && MMA_N % 64 == 0, "column tiling");
+constexpr int BN = 256;                 // columns per unit (one tcgen05.mma N)
 #ifndef SF_DW_BK
 #define SF_DW_BK 64
 #endif
@@ -64,18 +61,22 @@ constexpr int A_STAGE_BYTES = 4 * A_TILE_BYTES;    // 16 KB
 constexpr int B_BOX_BYTES = 64 * BK * 2;           // 64 columns x 64 tokens (128 B rows)
 constexpr int B_STAGE_BYTES = (BN / 64) * B_BOX_BYTES;   // 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-#ifndef SF_DW_NACC
-#define SF_DW_NACC 2
+// Accumulation in chunks. The tensor core adds each product block into its fp32 accumulator
+// with truncation, so over a long token sum the rounding errors share one sign and grow faster
+// than the sum (measured: ~T^1.5, a shrink toward zero). Each chunk of CHUNK tokens is therefore
+// summed by the MMAs into a TMEM buffer that starts from zero, and the epilogue adds the
+// finished chunks into fp32 registers with round-to-nearest. Two buffers let the MMAs fill one
+// while the epilogue drains the other.
+#ifndef SF_DW_CHUNK
+#define SF_DW_CHUNK 1024
 #endif
-#ifndef SF_DW_CTAS_PER_SM
-#define SF_DW_CTAS_PER_SM 1
-#endif
-constexpr int NACC = SF_DW_NACC;        // TMEM accumulators per CTA (the epilogue drains one while
-                                        // the MMAs fill the other)
-constexpr int kCtasPerSm = SF_DW_CTAS_PER_SM;
-constexpr int TMEM_COLS = NACC * BN;
-static_assert(NACC * kCtasPerSm * BN <= 512, "TMEM columns per SM");
-constexpr int kThreads = 192;
+constexpr int CHUNK_STAGES = SF_DW_CHUNK / BK;     // pipeline stages per accumulation chunk
+static_assert(SF_DW_CHUNK % BK == 0 && CHUNK_STAGES >= 1, "chunk of whole stages");
+constexpr int NBUF = 2;                 // TMEM chunk buffers
+constexpr int TMEM_COLS = NBUF * BN;    // 512: all of the SM's tensor memory (1 CTA per SM)
+constexpr int kEpiWarps = 8;            // two per TMEM lane quarter, one per 128-column half
+constexpr int kEpiCols = BN / 2;        // running sums per epilogue thread
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr size_t kSmemBytes = (size_t)STAGES * STAGE_BYTES + 1024;   // + alignment slack
 constexpr int kMaxPerGroup = 8;
 constexpr int kGatherTokens = 32;       // tokens per gather CTA
@@ -113,6 +114,7 @@ struct GatherProb {
     const int32_t *counts;
     const int32_t *row_slot;
     int64_t ld_dx;
+    int32_t R;
 };
 
 struct GatherGroup {
@@ -156,7 +158,7 @@ constexpr uint32_t kLayoutSW64 = 4;
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both MN-major, N, M.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                            ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 
 // Row mode when the group's active rows fit the scratch and need fewer 128-row tiles than the
 // mask tiles do. Every reader computes the same answer from the same counts.
@@ -169,10 +171,12 @@ __device__ __forceinline__ bool choose_rows(int rows, int tiles_mt, int mcap)
 // Row mode: dxg[t, k] = dX_p[t, r] for the group's k-th active row r (problems in call order,
 // rows ascending), and rowmap[k] = (slot(r) << 3) | p. One CTA per (group, 32 tokens); a thread
 // takes a gathered row and issues its 32 token loads back to back. The reads are single
-// elements spread over dX: each one costs the DRAM fetch of the line around it, so the loads
-// ask L2 for 64-byte fetches instead of the default 128 bytes (measured on the 7B step's
-// layout: ~57 instead of ~99 DRAM bytes per gathered element, the pass ~30% faster). Many
-// small independent loads per thread keep enough requests in flight.
+// elements spread over dX: each one costs the DRAM fetch of the line around it, so in a group
+// with fewer than one active row in 16 the loads ask L2 for 64-byte fetches instead of the
+// default 128 bytes (measured on the 7B step's layout at 1%: ~57 instead of ~99 DRAM bytes per
+// gathered element, the pass ~30% faster); denser groups use whole lines, which they need
+// anyway (64-byte fetches measured ~3x slower at 50%). Many small independent loads per thread
+// keep enough requests in flight.
 // Consecutive threads take consecutive gathered rows, so the writes coalesce. The first CTA of
 // a group records the mode and the row map, which the main kernel (next on the stream) reads.
 __global__ void __launch_bounds__(kGatherThreads)
@@ -182,17 +186,20 @@ dw_gather_kernel(const __grid_constant__ GatherBatch b, int blocks_per_group)
     const int tb = blockIdx.x - gi * blocks_per_group;
     const GatherGroup &g = b.g[gi];
     __shared__ int row_pre[kMaxPerGroup + 1];
-    __shared__ int s_rows_mode;
+    __shared__ int s_rows_mode, s_sparse;
     if (threadIdx.x == 0) {
         int rows = 0, tiles_mt = 0;
+        long long all_rows = 0;
         for (int k = 0; k < g.count; ++k) {
             const GatherProb &p = b.p[g.first + k];
             row_pre[k] = rows;
             rows += p.counts[0];
             tiles_mt += (p.counts[1] + 3) >> 2;
+            all_rows += p.R;
         }
         row_pre[g.count] = rows;
         s_rows_mode = choose_rows(rows, tiles_mt, g.mcap);
+        s_sparse = 16LL * rows < all_rows;             // fewer than 1 row in 16 active
         if (tb == 0) {
             g.info[0] = s_rows_mode;
             g.info[1] = rows;
@@ -216,9 +223,15 @@ dw_gather_kernel(const __grid_constant__ GatherBatch b, int blocks_per_group)
         const uint16_t *src = p.dx + (size_t)t0 * p.ld_dx + r;
         uint16_t *dst = g.dxg + (size_t)t0 * g.mcap + k;
         uint16_t v[kGatherTokens];
+        if (s_sparse) {
 #pragma unroll
-        for (int t = 0; t < kGatherTokens; ++t)
-            if (t < nt) v[t] = ld_nc_l2_64b_u16(src + (size_t)t * p.ld_dx);
+            for (int t = 0; t < kGatherTokens; ++t)
+                if (t < nt) v[t] = ld_nc_l2_64b_u16(src + (size_t)t * p.ld_dx);
+        } else {
+#pragma unroll
+            for (int t = 0; t < kGatherTokens; ++t)
+                if (t < nt) v[t] = __ldcs(src + (size_t)t * p.ld_dx);
+        }
 #pragma unroll
         for (int t = 0; t < kGatherTokens; ++t)
             if (t < nt) dst[(size_t)t * g.mcap] = v[t];
@@ -269,11 +282,11 @@ __device__ __forceinline__ Unit decode(int u, const SmemPlan &sp, const DwBatch 
 
 // ------------------------------------ main kernel ------------------------------------
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(kThreads, 1)
 masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
 {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2], tempty_bar[2], drain_bar;
+    __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[NBUF], tempty_bar[NBUF], drain_bar;
     __shared__ uint32_t tmem_base_s;
     __shared__ SmemPlan sp;
     __shared__ int scan_scratch[33];
@@ -312,9 +325,9 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
-        for (int a = 0; a < NACC; ++a) {
+        for (int a = 0; a < NBUF; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], 4);
+            mbar_init(&tempty_bar[a], kEpiWarps);
         }
         mbar_init(&drain_bar, 1);
         fence_mbarrier_init();
@@ -409,38 +422,37 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int acc = 0;
-            uint32_t acc_phase = 0;
+            int buf = 0;
+            uint32_t buf_phase = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
                 const Unit x = decode(u, sp, b);
                 const int nk = (grp(b, x.g).T + BK - 1) / BK;
-                if (nk == 0) continue;
-                if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, &abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < nk; ++kb) {
+                    const int in_chunk = kb % CHUNK_STAGES;
+                    if (in_chunk == 0) {             // a fresh chunk: wait until its buffer is drained
+                        if (!mbar_wait(&tempty_bar[buf], buf_phase ^ 1u, &abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                    }
                     if (!mbar_wait(&full_bar[stage], phase, &abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
                     const uint32_t sb = sa + A_STAGE_BYTES;
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
                         // 16 tokens = 16 rows of 64 B (A-operand) or 128 B (B-operand)
                         const uint64_t da = smem_desc(sa + k * UMMA_K * 64, A_TILE_BYTES, 8 * 64, kLayoutSW64);
-#pragma unroll
-                        for (int h = 0; h < NSUB; ++h) {
-                            const uint64_t db = smem_desc(sb + h * (MMA_N / 64) * B_BOX_BYTES + k * UMMA_K * 128,
-                                                          B_BOX_BYTES, 8 * 128, kLayoutSW128);
-                            mma_bf16(d_tmem + h * MMA_N, da, db, kIdesc, (kb | k) != 0);
-                        }
+                        const uint64_t db = smem_desc(sb + k * UMMA_K * 128, B_BOX_BYTES, 8 * 128, kLayoutSW128);
+                        mma_bf16(d_tmem, da, db, kIdesc, (in_chunk | k) != 0);
                     }
                     mma_commit(&empty_bar[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    if (in_chunk == CHUNK_STAGES - 1 || kb == nk - 1) {   // chunk complete
+                        mma_commit(&tfull_bar[buf]);
+                        if (++buf == NBUF) { buf = 0; buf_phase ^= 1u; }
+                    }
                 }
-                if (!ok) break;
-                mma_commit(&tfull_bar[acc]);
-                if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
             }
             // every MMA this thread issued has finished before TMEM is released
             mma_commit(&drain_bar);
@@ -448,10 +460,13 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
         }
     } else {
-        // ------------------------------ epilogue (warps 2..5) ------------------------------
+        // --------------------------- epilogue (warps 2..2+kEpiWarps-1) ---------------------------
+        // A warp may only read the TMEM lane quarter warp_id % 4; two warps share each quarter,
+        // one per 128-column half of the unit.
         const int quad = warp & 3;              // TMEM lanes 32*quad .. 32*quad+31
-        int acc = 0;
-        uint32_t acc_phase = 0;
+        const int half = (warp - 2) >> 2;       // columns half*128 .. half*128+127 of the unit
+        int buf = 0;
+        uint32_t buf_phase = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
             const Unit x = decode(u, sp, b);
             const DwGroup &g = grp(b, x.g);
@@ -473,38 +488,40 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 const int idx = x.mt * 4 + quad;
                 if (idx < p->counts[1]) slot = p->row_slot[p->active_tiles[idx] * 32 + lane];
             }
-            const int col_base = x.nt * BN;
+            const int col_base = x.nt * BN + half * kEpiCols;
             float *out = slot >= 0 ? p->dW + (size_t)slot * p->ld_dw : nullptr;
-            if (nk == 0) {                      // no tokens: the gradient is zero
-                if (out)
-                    for (int c = col_base; c < min(g.C, col_base + BN); c += 4)
-                        *reinterpret_cast<float4 *>(out + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-                continue;
-            }
-            // every lane waits; the outcome is made warp-uniform before the aligned TMEM loads
-            const bool ready = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, &abort_flag));
-            if (!ready) break;
-            tc_fence_after();
-            const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
-#pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(t_row + cc * 32, v);
-                tmem_ld_wait();
-                const int c0 = col_base + cc * 32;
-                if (out && c0 < g.C) {
+            float acc[kEpiCols];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        if (c0 + 4 * j < g.C)
-                            *reinterpret_cast<float4 *>(out + c0 + 4 * j) =
-                                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            for (int j = 0; j < kEpiCols; ++j) acc[j] = 0.0f;
+            bool ready = true;
+            const int nchunks = (nk + CHUNK_STAGES - 1) / CHUNK_STAGES;
+            for (int ch = 0; ch < nchunks; ++ch) {
+                // every lane waits; the outcome is made warp-uniform before the aligned TMEM loads
+                ready = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[buf], buf_phase, &abort_flag));
+                if (!ready) break;
+                tc_fence_after();
+                const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN + half * kEpiCols);
+#pragma unroll
+                for (int cc = 0; cc < kEpiCols / 32; ++cc) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(t_row + cc * 32, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[cc * 32 + j] = __fadd_rn(acc[cc * 32 + j], __uint_as_float(v[j]));
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+                if (++buf == NBUF) { buf = 0; buf_phase ^= 1u; }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-            if (++acc == NACC) { acc = 0; acc_phase ^= 1u; }
+            if (!ready) break;
+            if (out) {                          // no tokens: the sums stay zero, the gradient is zero
+#pragma unroll
+                for (int j = 0; j < kEpiCols / 4; ++j)
+                    if (col_base + 4 * j < g.C)
+                        *reinterpret_cast<float4 *>(out + col_base + 4 * j) =
+                            make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+            }
         }
     }
 
@@ -676,6 +693,7 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
                 d.counts = p.mask.counts;
                 d.row_slot = p.mask.row_slot;
                 d.ld_dx = p.ld_dx;
+                d.R = p.mask.R;
             }
         }
         if (gb->n_group > 0) {
@@ -757,7 +775,7 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
             max_units += tiles_mt * g.n_ntiles;
         }
         if (rc != SF_OK) break;
-        const int grid = (int)(max_units < (long long)sms * kCtasPerSm ? max_units : (long long)sms * kCtasPerSm);
+        const int grid = (int)(max_units < (long long)sms ? max_units : (long long)sms);
         if (grid > 0) {
             // launches after the first of the call overlap their predecessor's last wave
             cudaLaunchAttribute attr;
