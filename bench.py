@@ -37,6 +37,7 @@ METRIC = "sparse step ms & active-row updates/s at 7B shape, 1% active; % of roo
 TRAFFIC_PER_LAUNCH = {}
 TRAFFIC_NOTE = ""
 UNIT = "active-row updates/s"
+UNIT_ROWS = 256      # weight rows per dW tensor-core unit; main() sets it from the library
 SEED = 3
 SWEEP_SEED = 4
 
@@ -67,12 +68,12 @@ def parse():
                     help="layer chunks per step: chunk c's masks run on a side stream while earlier "
                          "chunks' dW and update run on the main stream (1, the default and the "
                          "fastest measured: one call per stage on one stream)")
-    ap.add_argument("--config", choices=["c0", "c1", "c2", "rewind"], default=None,
+    ap.add_argument("--config", choices=["c0", "c1", "c2", "rewind", "forward"], default=None,
                     help="time one of the smaller workloads instead of the headline step (one JSON line "
                          "each, not the headline metric): c0 the tiny projection, c1 the embedding "
                          "path, c2 one 7B-shaped layer at 4,096 tokens (scattered and clustered), rewind "
                          "the active-row checkpoint and a rewind-policy/Helix-driven run of the headline "
-                         "step")
+                         "step; forward the tracker folded into the forward projections' epilogue")
     ap.add_argument("--sweep", action="store_true",
                     help="density sweep of one 11008 x 4096 projection (T = 4096), scattered and "
                          "clustered rows, with a dense bf16 GEMM and a fused dense Adam as context; "
@@ -222,10 +223,10 @@ def step_work(model, counts, T):
     """counts: [n_mats, 8] host copy after a step. Returns the step's algorithmic work.
 
     Masked dW: per group, the device picks row mode when the group's active rows fit its scratch
-    (slot capacity rounded up to 32) and need fewer 128-row tiles than the mask tiles do; that
-    rule is mirrored here. Algorithmic bytes: A once per group, each active element of dX once
+    (slot capacity rounded up to 32) and need fewer units (UNIT_ROWS rows) than the mask tiles
+    do; that rule is mirrored here. Algorithmic bytes: A once per group, each active element of dX once
     (row mode) or each active mask tile of dX once (tile mode), each dW row written once. FLOPs:
-    useful = 2*T*C per active row; executed = 2*T*C*128 per 128-row tile.
+    useful = 2*T*C per active row; executed = 2*T*C*UNIT_ROWS per unit.
     """
     off = 1 if model.emb is not None else 0
     upd_bytes = 0
@@ -245,12 +246,12 @@ def step_work(model, counts, T):
         mats = [model.projs[i].mat for i in grp]
         cs = [counts[i + off] for i in grp]
         rows = sum(int(c[0]) for c in cs)
-        tiles_mt = sum((int(c[1]) + 3) // 4 for c in cs)
+        tiles_mt = sum(-(-int(c[1]) // (UNIT_ROWS // 32)) for c in cs)
         mcap = -(-sum(m.mask.slot_cap for m in mats) // 32) * 32
-        rows_mode = rows <= mcap and -(-rows // 128) < tiles_mt
-        mt = -(-rows // 128) if rows_mode else tiles_mt
+        rows_mode = rows <= mcap and -(-rows // UNIT_ROWS) < tiles_mt
+        mt = -(-rows // UNIT_ROWS) if rows_mode else tiles_mt
         C = mats[0].C
-        dw_flops_exec += mt * 128 * C * T * 2
+        dw_flops_exec += mt * UNIT_ROWS * C * T * 2
         dw_flops_useful += rows * C * T * 2
         a_and_rows = T * C * 2 + sum((int(c[0]) - int(c[3])) * C * 4 for c in cs)
         dx_once = T * rows * 2 if rows_mode else sum(int(c[1]) * 32 * T * 2 for c in cs)
@@ -452,10 +453,11 @@ def run_sweep(args):
             st /= steps
             cnt = mat.mask.counts.cpu().numpy()
             n_rows, n_tiles = int(cnt[0]), int(cnt[1])
-            mt_tiles = (n_tiles + 3) // 4
-            rows_mode = n_rows <= -(-cap // 32) * 32 and -(-n_rows // 128) < mt_tiles
-            mt = -(-n_rows // 128) if rows_mode else mt_tiles
-            dw_exec = mt * 128 * C * T * 2
+            um = sf.sf_masked_dw_unit_rows()
+            mt_tiles = -(-n_tiles // (um // 32))
+            rows_mode = n_rows <= -(-cap // 32) * 32 and -(-n_rows // um) < mt_tiles
+            mt = -(-n_rows // um) if rows_mode else mt_tiles
+            dw_exec = mt * um * C * T * 2
             dw_useful = n_rows * C * T * 2
             dw_bytes = T * C * 2 + n_rows * C * 4 + (T * n_rows * 2 if rows_mode else n_tiles * 32 * T * 2)
             upd_bytes = n_rows * C * 24 + n_rows * 8
@@ -697,6 +699,8 @@ def run_config(args):
     from masked_optimizer_step_b200 import synth
     from masked_optimizer_step_b200.model import INPUT_OF, Pipeline, SparseModel
     sf.load()
+    global UNIT_ROWS
+    UNIT_ROWS = sf.sf_masked_dw_unit_rows()
     device = "cuda:0"
     torch.cuda.set_device(0)
     stream = torch.cuda.current_stream()
@@ -780,6 +784,89 @@ def run_config(args):
     return 0
 
 
+def run_forward(args):
+    """The forward projections of the model with the row tracker folded into their epilogue
+    (sf_forward_tracked, then the masks' finalize), against the same forward projections as
+    cuBLAS bf16 GEMMs (torch.matmul) followed by the separate tracker pass (sf_mask_update, which
+    reads every Y again). Context for the fused kernel, not the headline metric."""
+    import torch
+    from masked_optimizer_step_b200 import binding as sf
+    from masked_optimizer_step_b200 import synth
+    from masked_optimizer_step_b200.model import INPUT_OF, SparseModel
+    sf.load()
+    device = "cuda:0"
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    T = args.tokens
+    model = SparseModel(args.layers, vocab=0, device=device)
+    model.init(SEED)
+    ins = {}
+    probs, Ys, srcs = [], [], []
+    for i, p in enumerate(model.projs):
+        key = (p.layer, INPUT_OF[p.name])
+        if key not in ins:
+            ins[key] = synth.device_normal_bf16((T, p.mat.C), SEED, "act", 7, p.layer, len(ins), device=device)
+        Y = torch.empty((T, p.mat.R), dtype=torch.bfloat16, device=device)
+        Ys.append(Y)
+        W = p.mat.live.view(torch.bfloat16)
+        probs.append(sf.fwd_problem(ins[key], W, Y, p.mat.mask))
+        srcs.append(sf.make_src(sf.SF_SRC_OUTPUT_BF16, Y, n=T, ld=Y.stride(0)))
+    masks = [p.mat.mask for p in model.projs]
+    flops = sum(2.0 * T * p.mat.R * p.mat.C for p in model.projs)
+    y_bytes = sum(T * p.mat.R * 2 for p in model.projs)
+    steps, warm = max(args.steps, 3), max(args.warmup, 3)
+
+    def fused():
+        sf.sf_forward_tracked(probs, None, stream)
+        sf.sf_mask_update_phase(masks, srcs, sf.SF_PHASE_SECOND, 0.01, None, stream)
+
+    def unfused():
+        for i, p in enumerate(model.projs):
+            torch.matmul(probs[i].refs[0], p.mat.live.view(torch.bfloat16).t(), out=Ys[i])
+        sf.sf_mask_update(masks, srcs, 0.01, None, stream)
+
+    def gemm_only():
+        for i, p in enumerate(model.projs):
+            torch.matmul(probs[i].refs[0], p.mat.live.view(torch.bfloat16).t(), out=Ys[i])
+
+    def fwd_only():
+        sf.sf_forward_tracked(probs, None, stream)
+
+    out = {}
+    for name, fn in (("fused", fused), ("unfused", unfused), ("cublas_gemm_only", gemm_only),
+                     ("fused_kernel_only", fwd_only)):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / steps
+    if "fused_kernel_only" in out:
+        # the accumulators took extra windows above: close them so the masks stay consistent
+        sf.sf_mask_update_phase(masks, srcs, sf.SF_PHASE_SECOND, 0.01, None, stream)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    tf = float(peaks.get("bf16_tflops", 1590.0))
+    line = {"config": "forward",
+            "workload": f"forward projections of {args.layers} 7B-shaped layers (7 each), {T} tokens, "
+                        "row tracker folded into the epilogue vs cuBLAS GEMM + separate tracker pass",
+            "ms": out, "gflop": flops / 1e9, "y_gb": y_bytes / 1e9,
+            "fused_kernel_tflops": flops / (out["fused_kernel_only"] / 1e3) / 1e12,
+            "fused_kernel_frac_of_bf16_burst": flops / (out["fused_kernel_only"] / 1e3) / 1e12 / tf,
+            "cublas_tflops": flops / (out["cublas_gemm_only"] / 1e3) / 1e12,
+            "tracker_pass_ms_saved": out["unfused"] - out["cublas_gemm_only"] - (out["fused"] - out["fused_kernel_only"]),
+            "fused_vs_unfused": out["unfused"] / out["fused"]}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -788,6 +875,8 @@ def main():
         return run_sweep(args)
     if args.config == "rewind":
         return run_rewind(args)
+    if args.config == "forward":
+        return run_forward(args)
     if args.config:
         return run_config(args)
     rank, world, local = dist_env()
@@ -802,6 +891,8 @@ def main():
     from masked_optimizer_step_b200 import binding as sf
     from masked_optimizer_step_b200.model import Pipeline, SparseModel
     sf.load()
+    global UNIT_ROWS
+    UNIT_ROWS = sf.sf_masked_dw_unit_rows()
 
     T = args.tokens
     model = SparseModel(n_layers=args.layers, device=device)
@@ -958,7 +1049,7 @@ def main():
                 "hbm_gbs": dw_gbs, "hbm_frac": dw_gbs / hbm,
                 "row_mode_groups_per_step": work[-1]["dw_row_groups"],
                 "algorithmic": "bytes: A once per group + active dX once + dW rows; FLOP: 2*T*C per "
-                               "executed row (128-row tiles)"}
+                               f"executed row ({UNIT_ROWS}-row units)"}
     step_bytes = trk_bytes + dw_bytes + upd_bytes
     stages = {
         "masks": {"ms_per_step": stage_ms[0] / args.steps, "bound": "hbm", "achieved": trk_gbs,
@@ -1006,7 +1097,7 @@ def main():
             kern["masked_dw_kernel"] = {"ms_per_step": main_s * 1e3 / K, "launches_per_step": plan0.dw_launches,
                                         "bound": "tensor", "algorithmic_flops_per_launch": dw_flops / K / plan0.dw_launches,
                                         "achieved": main_tf, "peak": tf_sus, "unit": "TFLOP/s", "frac": main_tf / tf_sus,
-                                        "algorithmic": "2*T*C FLOP per executed row (128-row tiles)"}
+                                        "algorithmic": f"2*T*C FLOP per executed row ({UNIT_ROWS}-row units)"}
         else:
             hbm_kernel("masked_dw_kernel", pass_ms["masked_dw:main"], main_bytes, plan0.dw_launches,
                        "A once per group + the gathered rows (row mode) or mask tiles of dX (tile mode) "

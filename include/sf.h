@@ -172,6 +172,12 @@ typedef struct sf_dw_problem {
 
 size_t sf_masked_dw_ws_bytes(const sf_dw_problem *probs /* host [n] */, int n);
 
+/* Weight rows per tensor-core unit of this build (256: a CTA pair's cta_group::2 MMA; 128: one
+ * CTA). A group runs in row mode when its active rows need fewer units than its mask tiles do
+ * (UNIT / 32 tiles per unit). Host-side mirrors of that choice (e.g. for counting the work) ask
+ * here. Needs no device. */
+int sf_masked_dw_unit_rows(void);
+
 int sf_masked_dw(const sf_dw_problem *probs /* host [n] */, int n, void *ws, size_t ws_bytes,
                  uint32_t *dev_status, sf_stream stream);
 
@@ -299,6 +305,37 @@ int sf_checkpoint_save(const sf_matrix *mats /* host [n] */, const sf_checkpoint
                        int n, uint32_t *dev_status, sf_stream stream);
 int sf_checkpoint_restore(const sf_matrix *mats /* host [n] */, const sf_checkpoint *ck /* host [n] */,
                           int n, uint32_t *dev_status, sf_stream stream);
+
+/* ---- sf_forward_tracked: section 2.1, the forward pass that the row tracker observes ---------
+ * A projection's activity for the charge rule is the magnitude of the outputs its forward pass
+ * produced. This call computes that forward pass and keeps the statistic on the way:
+ *     Y[t, r] = bf16_rn( sum_c A[t, c] * W[r, c] )     (fp32 accumulation, tensor cores)
+ * for every problem, stores Y, and folds max over its tokens of |Y[t, r]| (of the stored bf16
+ * values, with sf_mask_update's reading for non-finite outputs) into mask.accum[r] -- the same
+ * numbers sf_mask_update's SF_SRC_OUTPUT_BF16 pass would find by reading Y again. The window is
+ * then closed by sf_mask_update_phase(..., SF_PHASE_SECOND, ...) with an SF_SRC_OUTPUT_BF16
+ * source naming the same Y. Several calls may fold into one window before it is closed.
+ *   A  bf16 [T x ld_a]  the projection's inputs, token-major
+ *   W  bf16 [R x ld_w]  its weights (the bf16 live copy sf_sparse_update writes), row-major
+ *   Y  bf16 [T x ld_y]  its outputs (written)
+ * Requirements: R = mask.R a multiple of 32; C a multiple of 8; when T > 0, ld_a and ld_w
+ * multiples of 8 and >= C, ld_y a multiple of 8 and >= R, A, W, Y 16-byte aligned.
+ * Errors: SF_ERR_ARG, SF_ERR_ALIGN, SF_ERR_CUDA.
+ */
+typedef struct sf_fwd_problem {
+    const void *A;
+    int64_t     ld_a;
+    const void *W;
+    int64_t     ld_w;
+    void       *Y;
+    int64_t     ld_y;
+    int32_t     T;
+    int32_t     C;
+    sf_mask     mask;   /* R = mask.R; folds into mask.accum */
+} sf_fwd_problem;
+
+int sf_forward_tracked(const sf_fwd_problem *probs /* host [n] */, int n, uint32_t *dev_status,
+                       sf_stream stream);
 
 /* ---- sf_mask_update_phase / sf_masked_dw_phase: one pass of a two-pass call ------------------
  * No counterpart in the paper: a measurement aid. sf_mask_update and sf_masked_dw each run two

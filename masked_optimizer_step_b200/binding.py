@@ -57,6 +57,11 @@ class sf_dw_problem(ctypes.Structure):
                 ("mask", sf_mask), ("dW", _P), ("ld_dw", _I64)]
 
 
+class sf_fwd_problem(ctypes.Structure):
+    _fields_ = [("A", _P), ("ld_a", _I64), ("W", _P), ("ld_w", _I64), ("Y", _P), ("ld_y", _I64),
+                ("T", _I32), ("C", _I32), ("mask", sf_mask)]
+
+
 class sf_matrix(ctypes.Structure):
     _fields_ = [("C", _I32), ("partner", _I32), ("c_self", _F), ("c_partner", _F),
                 ("mask", sf_mask), ("q", _P), ("s", _P), ("delta", _P), ("m", _P), ("v", _P),
@@ -93,10 +98,13 @@ def load():
     L.sf_mask_update.argtypes = [ctypes.POINTER(sf_mask), ctypes.POINTER(sf_mask_src), ctypes.c_int,
                                  _F, _P, _P]
     L.sf_masked_dw.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int, _P, ctypes.c_size_t, _P, _P]
+    L.sf_forward_tracked.argtypes = [ctypes.POINTER(sf_fwd_problem), ctypes.c_int, _P, _P]
     L.sf_mask_update_phase.argtypes = [ctypes.POINTER(sf_mask), ctypes.POINTER(sf_mask_src), ctypes.c_int,
                                        _F, ctypes.c_int, _P, _P]
     L.sf_masked_dw_phase.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int, _P, ctypes.c_size_t,
                                      ctypes.c_int, _P, _P]
+    L.sf_masked_dw_unit_rows.restype = ctypes.c_int
+    L.sf_masked_dw_unit_rows.argtypes = []
     L.sf_masked_dw_ws_bytes.restype = ctypes.c_size_t
     L.sf_masked_dw_ws_bytes.argtypes = [ctypes.POINTER(sf_dw_problem), ctypes.c_int]
     L.sf_embed_grad_ws_bytes.restype = ctypes.c_size_t
@@ -114,7 +122,8 @@ def load():
         getattr(L, name).argtypes = [ctypes.POINTER(sf_matrix), ctypes.POINTER(sf_checkpoint), ctypes.c_int, _P, _P]
         getattr(L, name).restype = ctypes.c_int
     for name in ("sf_mask_init", "sf_mask_update", "sf_masked_dw", "sf_embed_grad", "sf_adam_tables",
-                 "sf_sparse_update", "sf_quantize_init", "sf_mask_update_phase", "sf_masked_dw_phase"):
+                 "sf_sparse_update", "sf_quantize_init", "sf_mask_update_phase", "sf_masked_dw_phase",
+                 "sf_forward_tracked"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -246,6 +255,10 @@ def dw_problem(dX, A, mask: Mask, dW) -> Desc:
     return Desc(c, dX, A, dW)
 
 
+def sf_masked_dw_unit_rows() -> int:
+    return load().sf_masked_dw_unit_rows()
+
+
 def sf_masked_dw_ws_bytes(problems) -> int:
     n = len(problems)
     arr = (sf_dw_problem * n)(*[p.c for p in problems])
@@ -273,6 +286,24 @@ def sf_masked_dw_phase(problems, phase: int, status=None, stream=None, ws=None):
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(load().sf_masked_dw_phase(arr, n, _ptr(ws), nbytes, phase, _ptr(status), _stream(stream)),
            "sf_masked_dw_phase")
+
+
+def fwd_problem(A, W, Y, mask: Mask) -> Desc:
+    """A [T x C] bf16 inputs, W [R x C] bf16 weights, Y [T x R] bf16 outputs (written)."""
+    T, C = A.shape
+    R = W.shape[0]
+    assert W.shape[1] == C and Y.shape == (T, R) and R == mask.R
+    assert A.dtype == W.dtype == Y.dtype == torch.bfloat16
+    c = sf_fwd_problem(_ptr(A), A.stride(0), _ptr(W), W.stride(0), _ptr(Y), Y.stride(0), T, C, mask.struct())
+    return Desc(c, A, W, Y)
+
+
+def sf_forward_tracked(problems, status=None, stream=None):
+    """Forward projections Y = A W^T with each projection's row magnitudes folded into its mask's
+    accumulator; close the window with sf_mask_update_phase(..., SF_PHASE_SECOND)."""
+    n = len(problems)
+    arr = (sf_fwd_problem * max(n, 1))(*[p.c for p in problems])
+    _check(load().sf_forward_tracked(arr, n, _ptr(status), _stream(stream)), "sf_forward_tracked")
 
 
 def sf_embed_grad_ws_bytes(n_tok: int, slot_cap: int) -> int:

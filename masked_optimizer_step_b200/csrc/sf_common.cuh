@@ -190,6 +190,20 @@ SF_DEVICE void tma_load_2d(void *dst, const CUtensorMap *m, uint64_t *bar, int x
         : "memory");
 }
 
+// 2-D tiled TMA load by either CTA of a pair into its own shared memory, completing its bytes on
+// the mbarrier at `bar`'s offset in the even CTA (the one whose thread issues the pair's MMAs).
+// No multicast.
+SF_DEVICE void tma_load_2d_pair(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y)
+{
+    asm volatile(
+        "{\n\t.reg .b32 rb;\n\t"
+        "mapa.shared::cluster.u32 rb, %2, 0;\n\t"
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [rb];\n\t}"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
 SF_DEVICE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 SF_DEVICE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -245,5 +259,68 @@ SF_DEVICE void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32])
 }
 
 SF_DEVICE void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// --------------------------------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs sharing one tcgen05.mma with cta_group::2).
+// --------------------------------------------------------------------------------------------
+
+SF_DEVICE uint32_t cluster_ctarank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of the cluster.
+SF_DEVICE void mbar_arrive_remote(uint64_t *bar, uint32_t rank)
+{
+    asm volatile("{\n\t.reg .b32 ra;\n\t"
+                 "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+                 "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+                 ::"r"(smem_u32(bar)), "r"(rank) : "memory");
+}
+
+// Every thread of every CTA of the cluster arrives, then waits for all of them.
+SF_DEVICE void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// TMEM allocation for a CTA pair: issued by the same warp of both CTAs, same destination offset.
+SF_DEVICE void tmem_alloc_pair(uint32_t *dst, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(dst)), "r"(ncols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+SF_DEVICE void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// D[tmem] (+)= A * B over the CTA pair (M = 256: 128 rows of A and N/2 columns of B in each
+// CTA's shared memory, at the same offsets), issued by one thread of the even CTA.
+SF_DEVICE void mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                             uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the mbarrier at `bar`'s offset in every CTA of `mask` once the pair's tcgen05
+// operations issued so far by this thread have completed.
+SF_DEVICE void mma_commit_pair(uint64_t *bar, uint16_t mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(smem_u32(bar)), "h"(mask) : "memory");
+}
 
 }  // namespace sf

@@ -44,8 +44,22 @@
 namespace sf {
 namespace {
 
-constexpr int BM = 128;                 // rows per unit
+constexpr int BM = 128;                 // rows per CTA of a unit (TMEM lanes)
 constexpr int BN = 256;                 // columns per unit (one tcgen05.mma N)
+#ifndef SF_DW_PAIR
+#define SF_DW_PAIR 1
+#endif
+// CTAs sharing a unit: with 2, a cluster pair runs one tcgen05.mma with cta_group::2 (M = 256):
+// each CTA loads its own 128 rows and its own half of the unit's columns (completing on the
+// even CTA's barriers), so the shared-memory traffic per FLOP is two thirds of a single CTA's.
+// Measured on B200 (parity green in both builds): no faster on dense masks (50% of rows:
+// 186 vs 182 us for one 11008 x 4096 projection at 4,096 tokens) and 24% slower on the 7B step's
+// scattered 1% masks (0.82 vs 0.66 ms), so one CTA per unit is the default.
+constexpr int PAIR = SF_DW_PAIR;
+static_assert(PAIR == 1 || PAIR == 2, "one CTA or a CTA pair per unit");
+constexpr int UM = BM * PAIR;           // rows per unit
+constexpr int UNIT_TILES = UM / 32;     // 32-row mask tiles per unit (tile mode)
+constexpr int B_COLS = BN / PAIR;       // columns of the unit each CTA loads
 #ifndef SF_DW_BK
 #define SF_DW_BK 64
 #endif
@@ -53,13 +67,13 @@ constexpr int BK = SF_DW_BK;            // tokens per pipeline stage
 constexpr int UMMA_K = 16;              // K of one tcgen05.mma kind::f16
 static_assert(BK % UMMA_K == 0 && BK <= 256, "stage depth");
 #ifndef SF_DW_STAGES
-#define SF_DW_STAGES 4
+#define SF_DW_STAGES (PAIR == 2 ? 6 : 4)
 #endif
 constexpr int STAGES = SF_DW_STAGES;
 constexpr int A_TILE_BYTES = 32 * BK * 2;          // 32 rows x 64 tokens (64 B rows)
 constexpr int A_STAGE_BYTES = 4 * A_TILE_BYTES;    // 16 KB
 constexpr int B_BOX_BYTES = 64 * BK * 2;           // 64 columns x 64 tokens (128 B rows)
-constexpr int B_STAGE_BYTES = (BN / 64) * B_BOX_BYTES;   // 32 KB
+constexpr int B_STAGE_BYTES = (B_COLS / 64) * B_BOX_BYTES;   // 16 KB (pair) or 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 // Accumulation in chunks. The tensor core adds each product block into its fp32 accumulator
 // with truncation, so over a long token sum the rounding errors share one sign and grow faster
@@ -158,13 +172,13 @@ constexpr uint32_t kLayoutSW64 = 4;
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both MN-major, N, M.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(UM >> 4) << 24);
 
-// Row mode when the group's active rows fit the scratch and need fewer 128-row tiles than the
-// mask tiles do. Every reader computes the same answer from the same counts.
+// Row mode when the group's active rows fit the scratch and need fewer units than the mask
+// tiles do. Every reader computes the same answer from the same counts.
 __device__ __forceinline__ bool choose_rows(int rows, int tiles_mt, int mcap)
 {
-    return mcap > 0 && rows <= mcap && (rows + BM - 1) / BM < tiles_mt;
+    return mcap > 0 && rows <= mcap && (rows + UM - 1) / UM < tiles_mt;
 }
 
 // ------------------------------------ gather kernel ------------------------------------
@@ -194,7 +208,7 @@ dw_gather_kernel(const __grid_constant__ GatherBatch b, int blocks_per_group)
             const GatherProb &p = b.p[g.first + k];
             row_pre[k] = rows;
             rows += p.counts[0];
-            tiles_mt += (p.counts[1] + 3) >> 2;
+            tiles_mt += (p.counts[1] + UNIT_TILES - 1) / UNIT_TILES;
             all_rows += p.R;
         }
         row_pre[g.count] = rows;
@@ -285,6 +299,12 @@ __device__ __forceinline__ Unit decode(int u, const SmemPlan &sp, const DwBatch 
 __global__ void __launch_bounds__(kThreads, 1)
 masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
 {
+    // CTA pairs: the even CTA of a cluster (the leader) issues the MMAs of both and owns the
+    // stage barriers; the odd one loads its halves (completing on the leader's barriers) and
+    // drains its own TMEM lanes.
+    const uint32_t crank = PAIR == 2 ? cluster_ctarank() : 0u;
+    const bool leader = crank == 0;
+    const int unit0 = blockIdx.x / PAIR, ustep = gridDim.x / PAIR;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[NBUF], tempty_bar[NBUF], drain_bar;
     __shared__ uint32_t tmem_base_s;
@@ -308,11 +328,11 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             int acc = 0;
             for (int k = 0; k < g.count; ++k) {
                 sp.mt_prefix[g.first + k] = acc;
-                acc += (prb(b, g.first + k).counts[1] + 3) >> 2;
+                acc += (prb(b, g.first + k).counts[1] + UNIT_TILES - 1) / UNIT_TILES;
             }
             const int rows_mode = g.info != nullptr && g.info[0] != 0;
             sp.rows_mode[tid] = rows_mode;
-            units = (rows_mode ? (g.info[1] + BM - 1) / BM : acc) * g.n_ntiles;
+            units = (rows_mode ? (g.info[1] + UM - 1) / UM : acc) * g.n_ntiles;
         }
         int total;
         const int off = block_exclusive_scan(units, scan_scratch, &total);
@@ -322,19 +342,24 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
     if (tid == 0) {
         abort_flag = 0;
         for (int s = 0; s < STAGES; ++s) {
+            // in a pair only the leader's full barriers are used: both CTAs' loads complete on them
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
         for (int a = 0; a < NBUF; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], kEpiWarps);
+            mbar_init(&tempty_bar[a], kEpiWarps * PAIR);    // the leader's counts both CTAs' warps
         }
         mbar_init(&drain_bar, 1);
         fence_mbarrier_init();
     }
-    if (warp == 1) tmem_alloc(&tmem_base_s, TMEM_COLS);
+    if (warp == 1) {
+        if (PAIR == 2) tmem_alloc_pair(&tmem_base_s, TMEM_COLS);
+        else tmem_alloc(&tmem_base_s, TMEM_COLS);
+    }
     tc_fence_before();
     __syncthreads();
+    if (PAIR == 2) cluster_sync();            // both CTAs' barriers exist before either uses them
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_s;
     const int total_units = sp.unit_prefix[b.n_group];
@@ -351,7 +376,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             bool issued[STAGES] = {};
             uint32_t issued_parity[STAGES] = {};
             bool ok = true;
-            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+            for (int u = unit0; u < total_units && ok; u += ustep) {
                 const Unit x = decode(u, sp, b);
                 const DwGroup &g = grp(b, x.g);
                 const int nk = (g.T + BK - 1) / BK;
@@ -363,7 +388,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     const int total = g.info[1];
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
-                        const int k0 = x.mt * BM + s * 32;
+                        const int k0 = x.mt * UM + (int)crank * BM + s * 32;
                         coord[s] = k0 < total ? k0 : -1;
                         nvalid += coord[s] >= 0;
                     }
@@ -373,29 +398,43 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     const int n_tiles = p.counts[1];
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
-                        const int idx = x.mt * 4 + s;
+                        const int idx = x.mt * UNIT_TILES + (int)crank * 4 + s;
                         coord[s] = idx < n_tiles ? p.active_tiles[idx] * 32 : -1;
                         nvalid += coord[s] >= 0;
                     }
                 }
-                const uint32_t bytes = nvalid * A_TILE_BYTES + B_STAGE_BYTES;
+                // the leader's barrier counts both CTAs' bytes: the peer's boxes are the next four
+                // tiles (or gathered rows) of the unit
+                int nvalid_peer = 0;
+                if (PAIR == 2 && leader) {
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        if (x.rows_mode) nvalid_peer += x.mt * UM + BM + s * 32 < g.info[1];
+                        else nvalid_peer += x.mt * UNIT_TILES + 4 + s < prb(b, x.p).counts[1];
+                    }
+                }
+                const uint32_t bytes = (nvalid + nvalid_peer) * A_TILE_BYTES + PAIR * B_STAGE_BYTES;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { ok = false; break; }
                     uint8_t *sa = smem + stage * STAGE_BYTES;
                     uint8_t *sb = sa + A_STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                    if (leader) mbar_arrive_expect_tx(&full_bar[stage], PAIR == 2 ? bytes : nvalid * A_TILE_BYTES + B_STAGE_BYTES);
                     // test hook (failure detection): the stage's bytes never arrive, so the MMA
                     // issuer's bounded wait runs out and the CTA unwinds with WAIT_TIMEOUT
-                    const bool withhold = b.withhold_test && blockIdx.x == 0 && u == (int)blockIdx.x && kb == 0;
+                    const bool withhold = b.withhold_test && blockIdx.x == 0 && u == unit0 && kb == 0;
                     if (!withhold) {
 #pragma unroll
                         for (int s = 0; s < 4; ++s)
-                            if (coord[s] >= 0)
-                                tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
+                            if (coord[s] >= 0) {
+                                if (PAIR == 2) tma_load_2d_pair(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
+                                else tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
+                            }
 #pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            tma_load_2d(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], x.nt * BN + j * 64,
-                                        kb * BK);
+                        for (int j = 0; j < B_COLS / 64; ++j) {
+                            const int col = x.nt * BN + (int)crank * B_COLS + j * 64;
+                            if (PAIR == 2) tma_load_2d_pair(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], col, kb * BK);
+                            else tma_load_2d(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], col, kb * BK);
+                        }
                     }
                     issued[stage] = true;
                     issued_parity[stage] = phase;
@@ -407,8 +446,9 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
             }
-            if (!ok || abort_flag) {
-                // drain this CTA's own loads before the shared memory goes away
+            if ((!ok || abort_flag) && leader) {
+                // drain the loads armed on this CTA's barriers before the shared memory goes away
+                // (in a pair both CTAs' loads complete on the leader's barriers)
                 for (int s = 0; s < STAGES; ++s) {
                     if (!issued[s]) continue;
                     const uint64_t t0 = globaltimer_ns();
@@ -417,6 +457,8 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 }
             }
         }
+    } else if (warp == 1 && PAIR == 2 && !leader) {
+        // the odd CTA of a pair issues no MMAs: the leader's thread issues them for both
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
@@ -425,7 +467,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             int buf = 0;
             uint32_t buf_phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+            for (int u = unit0; u < total_units && ok; u += ustep) {
                 const Unit x = decode(u, sp, b);
                 const int nk = (grp(b, x.g).T + BK - 1) / BK;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -444,18 +486,22 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                         // 16 tokens = 16 rows of 64 B (A-operand) or 128 B (B-operand)
                         const uint64_t da = smem_desc(sa + k * UMMA_K * 64, A_TILE_BYTES, 8 * 64, kLayoutSW64);
                         const uint64_t db = smem_desc(sb + k * UMMA_K * 128, B_BOX_BYTES, 8 * 128, kLayoutSW128);
-                        mma_bf16(d_tmem, da, db, kIdesc, (in_chunk | k) != 0);
+                        if (PAIR == 2) mma_bf16_pair(d_tmem, da, db, kIdesc, (in_chunk | k) != 0);
+                        else mma_bf16(d_tmem, da, db, kIdesc, (in_chunk | k) != 0);
                     }
-                    mma_commit(&empty_bar[stage]);
+                    if (PAIR == 2) mma_commit_pair(&empty_bar[stage], 3);   // both CTAs' stages free
+                    else mma_commit(&empty_bar[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                     if (in_chunk == CHUNK_STAGES - 1 || kb == nk - 1) {   // chunk complete
-                        mma_commit(&tfull_bar[buf]);
+                        if (PAIR == 2) mma_commit_pair(&tfull_bar[buf], 3);
+                        else mma_commit(&tfull_bar[buf]);
                         if (++buf == NBUF) { buf = 0; buf_phase ^= 1u; }
                     }
                 }
             }
             // every MMA this thread issued has finished before TMEM is released
-            mma_commit(&drain_bar);
+            if (PAIR == 2) mma_commit_pair(&drain_bar, 3);
+            else mma_commit(&drain_bar);
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
         }
@@ -467,7 +513,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
         const int half = (warp - 2) >> 2;       // columns half*128 .. half*128+127 of the unit
         int buf = 0;
         uint32_t buf_phase = 0;
-        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+        for (int u = unit0; u < total_units; u += ustep) {
             const Unit x = decode(u, sp, b);
             const DwGroup &g = grp(b, x.g);
             const int nk = (g.T + BK - 1) / BK;
@@ -475,7 +521,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             int slot = -1;
             const DwProb *p = nullptr;
             if (x.rows_mode) {
-                const int k = x.mt * BM + quad * 32 + lane;
+                const int k = x.mt * UM + (int)crank * BM + quad * 32 + lane;
                 if (k < g.info[1]) {
                     const int e = g.rowmap[k];
                     if (e >= 0) {
@@ -485,7 +531,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 }
             } else {
                 p = &prb(b, x.p);
-                const int idx = x.mt * 4 + quad;
+                const int idx = x.mt * UNIT_TILES + (int)crank * 4 + quad;
                 if (idx < p->counts[1]) slot = p->row_slot[p->active_tiles[idx] * 32 + lane];
             }
             const int col_base = x.nt * BN + half * kEpiCols;
@@ -511,7 +557,10 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+                if (lane == 0) {                 // the leader's MMAs may refill the buffer
+                    if (PAIR == 2 && !leader) mbar_arrive_remote(&tempty_bar[buf], 0);
+                    else mbar_arrive(&tempty_bar[buf]);
+                }
                 if (++buf == NBUF) { buf = 0; buf_phase ^= 1u; }
             }
             if (!ready) break;
@@ -528,10 +577,12 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
     __syncwarp();                       // lanes 1..31 of the producer and MMA warps rejoin lane 0
     tc_fence_before();
     __syncthreads();
+    if (PAIR == 2) cluster_sync();            // neither CTA leaves while the pair's MMAs may run
     if (abort_flag && tid == 0) set_status(status, SF_STATUS_WAIT_TIMEOUT);
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if (PAIR == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
     // Complete only after the launch before this one has: whatever the stream runs next then
     // sees every launch of the call finished.
@@ -618,6 +669,8 @@ size_t launch_bytes(const HostGroup &g) { return sizeof(DwGroup) + (size_t)g.cou
 
 using namespace sf;
 
+extern "C" int sf_masked_dw_unit_rows(void) { return UM; }
+
 extern "C" size_t sf_masked_dw_ws_bytes(const sf_dw_problem *probs, int n)
 {
     if (n <= 0 || !probs) return 0;
@@ -663,6 +716,22 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
     if (rc == SF_OK && cudaFuncSetAttribute(masked_dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             (int)kSmemBytes) != cudaSuccess)
         rc = SF_ERR_CUDA;
+    int pair_slots = 0;                       // CTA pairs that can be resident at once
+    if (rc == SF_OK && PAIR == 2 && phase != SF_PHASE_FIRST) {
+        cudaLaunchConfig_t qcfg = {};
+        cudaLaunchAttribute qattr;
+        qattr.id = cudaLaunchAttributeClusterDimension;
+        qattr.val.clusterDim.x = 2;
+        qattr.val.clusterDim.y = 1;
+        qattr.val.clusterDim.z = 1;
+        qcfg.gridDim = dim3(2 * sms);
+        qcfg.blockDim = dim3(kThreads);
+        qcfg.dynamicSmemBytes = kSmemBytes;
+        qcfg.attrs = &qattr;
+        qcfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&pair_slots, masked_dw_kernel, &qcfg) != cudaSuccess || pair_slots <= 0)
+            rc = SF_ERR_CUDA;
+    }
     cudaStream_t st = as_stream(stream);
     auto scratch = [&](const HostGroup &hg) { return static_cast<uint8_t *>(ws) + hg.ws_off; };
     auto row_ok = [&](const HostGroup &hg) { return use_ws && probs[hg.first].T > 0 && hg.mcap > 0; };
@@ -770,24 +839,36 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
                 d.row_slot = p.mask.row_slot;
                 d.dW = p.dW;
                 d.ld_dw = p.ld_dw;
-                tiles_mt += (p.mask.R / 32 + 3) / 4;
+                tiles_mt += (p.mask.R / 32 + UNIT_TILES - 1) / UNIT_TILES;
             }
             max_units += tiles_mt * g.n_ntiles;
         }
         if (rc != SF_OK) break;
-        const int grid = (int)(max_units < (long long)sms ? max_units : (long long)sms);
+        const long long slots = PAIR == 2 ? (long long)pair_slots : (long long)sms;
+        const int grid = PAIR * (int)(max_units < slots ? max_units : slots);
         if (grid > 0) {
             // launches after the first of the call overlap their predecessor's last wave
-            cudaLaunchAttribute attr;
-            attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr.val.programmaticStreamSerializationAllowed = 1;
+            cudaLaunchAttribute attr[2];
+            int na = 0;
+            if (PAIR == 2) {
+                attr[na].id = cudaLaunchAttributeClusterDimension;
+                attr[na].val.clusterDim.x = 2;
+                attr[na].val.clusterDim.y = 1;
+                attr[na].val.clusterDim.z = 1;
+                ++na;
+            }
+            if (n_main_launches > 0) {
+                attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                attr[na].val.programmaticStreamSerializationAllowed = 1;
+                ++na;
+            }
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(grid);
             cfg.blockDim = dim3(kThreads);
             cfg.dynamicSmemBytes = kSmemBytes;
             cfg.stream = st;
-            cfg.attrs = &attr;
-            cfg.numAttrs = n_main_launches > 0 ? 1 : 0;
+            cfg.attrs = attr;
+            cfg.numAttrs = na;
             if (cudaLaunchKernelEx(&cfg, masked_dw_kernel, *batch, dev_status) != cudaSuccess ||
                 launch_status() != SF_OK) {
                 rc = SF_ERR_CUDA;

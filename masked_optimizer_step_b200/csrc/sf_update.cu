@@ -25,7 +25,10 @@
 namespace sf {
 namespace {
 
-constexpr int kThreads = 256;
+#ifndef SF_UPDATE_THREADS
+#define SF_UPDATE_THREADS 256
+#endif
+constexpr int kThreads = SF_UPDATE_THREADS;     // threads per CTA (one row at a time)
 constexpr int kMaxMatsPerLaunch = 256;
 constexpr int kMaxC = 32768;
 
@@ -163,7 +166,7 @@ __device__ __forceinline__ void adam_chunk(const Chunk &k, const AdamRow &a, flo
 // once and parks the new fp32 weight in shared memory (4*C bytes), so a thread needs few
 // registers and several CTAs share an SM; pass 2 requantises from shared memory.
 template <int UNROLL>
-__global__ void __launch_bounds__(kThreads, UNROLL == 1 ? 4 : 3)
+__global__ void __launch_bounds__(kThreads, (UNROLL == 1 ? 1024 : 768) / kThreads)
 update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
 {
     extern __shared__ float4 wrow4[];                 // new weights of the current row

@@ -228,6 +228,17 @@ def masked_dw_rows(dX_bf16: np.ndarray, A_bf16: np.ndarray, rows) -> np.ndarray:
     return wide(dX[:, rows]).T @ wide(A)
 
 
+def forward_product(A_bf16: np.ndarray, W_bf16: np.ndarray) -> np.ndarray:
+    """Y = A W^T in fp64 (A [T x C], W [R x C], bf16 bits), the forward projection whose output
+    magnitudes the row tracker observes (section 2.1). The bf16 inputs widen exactly; the fp64
+    matrix product of numpy is the summation step."""
+    A = _arr(A_bf16, np.uint16)
+    W = _arr(W_bf16, np.uint16)
+    assert A.shape[1] == W.shape[1]
+    wide = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return wide(A) @ wide(W).T
+
+
 def embed_grad(tokens, dY_bf16: np.ndarray, V: int, words: np.ndarray,
                out: np.ndarray | None = None) -> np.ndarray:
     """G[r] = sum of dY rows of the tokens with id r, active rows only (fp64)."""

@@ -68,7 +68,7 @@ def _c_struct_fields(name):
 
 
 @pytest.mark.parametrize("name", ["sf_mask", "sf_mask_src", "sf_dw_problem", "sf_matrix", "sf_adam",
-                                  "sf_checkpoint"])
+                                  "sf_checkpoint", "sf_fwd_problem"])
 def test_binding_structs_follow_the_header(name):
     py = [f[0] for f in getattr(binding, name)._fields_]
     assert py == _c_struct_fields(name)

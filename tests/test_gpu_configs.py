@@ -294,7 +294,8 @@ def test_c4_density_point_matches_oracle(sf, kind, density):
     check_slot_invariants(mh, cap)
 
     # the device picks row mode when the gathered rows need fewer tensor-core tiles
-    rows_mode = -(-len(rows) // 128) < -(-len(tiles) // 4) and len(rows) <= -(-cap // 32) * 32
+    um = sf.sf_masked_dw_unit_rows()
+    rows_mode = -(-len(rows) // um) < -(-len(tiles) // (um // 32)) and len(rows) <= -(-cap // 32) * 32
     assert rows_mode == (kind == "scattered")
     per_tile = _rows_per_tc_tile(rows, tiles, rows_mode)
     assert len(per_tile) >= 5

@@ -235,6 +235,24 @@ def test_activity_rule_split_over_token_shares():
     assert c3.tobytes() == (np.float32(0.5) * c1).tobytes()
 
 
+def test_forward_product_matches_brute_force():
+    # integer-valued bf16 inputs keep fp64 sums exact: the product must equal the plain triple
+    # loop bit for bit, and a transposed operand must not
+    g = np.random.default_rng(13)
+    T, C, R = 7, 24, 5
+    A = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(T, C)).astype(np.float32))
+    W = synth.f32_to_bf16_bits(g.integers(-8, 9, size=(R, C)).astype(np.float32))
+    Af, Wf = synth.bf16_bits_to_f32(A), synth.bf16_bits_to_f32(W)
+    ref = np.zeros((T, R))
+    for t in range(T):
+        for r in range(R):
+            for c in range(C):
+                ref[t, r] += float(Af[t, c]) * float(Wf[r, c])
+    got = orc.forward_product(A, W)
+    assert got.shape == (T, R) and np.array_equal(got, ref)
+    assert not np.array_equal(orc.forward_product(A[:, ::-1], W), ref)
+
+
 def test_tracker_recipe_turns_exactly_the_chosen_rows_on():
     g = synth.rng(2, "tracker", 0)
     R, T = 1024, 512
