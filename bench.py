@@ -34,8 +34,13 @@ METRIC = "sparse step ms & active-row updates/s at 7B shape, 1% active; % of roo
 # DRAM traffic per launch of a kernel (dram__bytes_read.sum + dram__bytes_write.sum from one ncu
 # capture), keyed by (layers, tokens, masks) of the workload it was captured on; a kernel or
 # workload not listed has none. Entries are removed whenever the kernel changes.
-TRAFFIC_PER_LAUNCH = {}
-TRAFFIC_NOTE = ""
+TRAFFIC_PER_LAUNCH = {
+    "mask_accum_kernel": {(32, 2048, "scattered"): 16 * 348.7e6},
+    "dw_gather_kernel": {(32, 2048, "scattered"): 16 * 101.5e6},
+}
+TRAFFIC_NOTE = ("ncu DRAM bytes of the 2-layer case of this workload (profiles/kernels_2layer_dram.md) "
+                "scaled by 16 to 32 layers: one launch per step either way, bytes in proportion to the "
+                "layers")
 UNIT = "active-row updates/s"
 UNIT_ROWS = 256      # weight rows per dW tensor-core unit; main() sets it from the library
 SEED = 3

@@ -204,6 +204,30 @@ SF_DEVICE void tma_load_2d_pair(void *dst, const CUtensorMap *m, uint64_t *bar, 
         : "memory");
 }
 
+// 3-D tiled TMA load of box {x, y, z} into shared memory (box element order x fastest, then y,
+// then z), completing transaction bytes on `bar`. No multicast.
+SF_DEVICE void tma_load_3d(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y, int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z),
+          "r"(smem_u32(bar))
+        : "memory");
+}
+
+// The CTA-pair form of tma_load_3d (completing on the even CTA's barrier). No multicast.
+SF_DEVICE void tma_load_3d_pair(void *dst, const CUtensorMap *m, uint64_t *bar, int x, int y, int z)
+{
+    asm volatile(
+        "{\n\t.reg .b32 rb;\n\t"
+        "mapa.shared::cluster.u32 rb, %2, 0;\n\t"
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [rb];\n\t}"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
 SF_DEVICE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 SF_DEVICE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 

@@ -106,11 +106,16 @@ struct alignas(64) DwProb {
 };
 
 struct alignas(64) DwGroup {
-    CUtensorMap tm_a;            // A: dims {C, T}, box {64, 64}, 128-byte swizzle
-    CUtensorMap tm_g;            // gathered rows: dims {mcap, T}, box {32, 64}, 64-byte swizzle
+    // A: when C is a multiple of 64, 3-D {64 columns, T, C / 64 chunks} with box {64, 64,
+    // B_COLS / 64}: one load brings the CTA's column chunks of a stage, chunk after chunk (the
+    // layout the four 2-D boxes give); otherwise 2-D {C, T}, box {64, 64}. 128-byte swizzle.
+    CUtensorMap tm_a;
+    // gathered rows: 3-D {32 rows, T, mcap / 32 chunks}, box {32, 64, 4}, 64-byte swizzle (or
+    // 2-D {mcap, T}, box {32, 64}, when the 3-D map is not accepted)
+    CUtensorMap tm_g;
     const int32_t *info;         // device: [0] mode (1 = rows), [1] gathered rows (null: tiles only)
     const int32_t *rowmap;       // device: per gathered row, (slot << 3) | problem, or -1
-    int32_t first, count, C, T, n_ntiles, mcap;
+    int32_t first, count, C, T, n_ntiles, mcap, a3d, g3d;   // g3d: tm_g is 3-D (else 2-D, box {32, 64})
 };
 
 struct DwBatch {
@@ -383,7 +388,12 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 const CUtensorMap *tm_rows;
                 int coord[4];
                 int nvalid = 0;
-                if (x.rows_mode) {
+                if (x.rows_mode && g.g3d) {         // one 3-D box: the CTA's four 32-row chunks
+                    tm_rows = &g.tm_g;
+                    coord[0] = (x.mt * UM + (int)crank * BM) / 32;
+                    coord[1] = coord[2] = coord[3] = -1;
+                    nvalid = 4;
+                } else if (x.rows_mode) {
                     tm_rows = &g.tm_g;
                     const int total = g.info[1];
 #pragma unroll
@@ -409,7 +419,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 if (PAIR == 2 && leader) {
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
-                        if (x.rows_mode) nvalid_peer += x.mt * UM + BM + s * 32 < g.info[1];
+                        if (x.rows_mode) nvalid_peer += g.g3d || x.mt * UM + BM + s * 32 < g.info[1];
                         else nvalid_peer += x.mt * UNIT_TILES + 4 + s < prb(b, x.p).counts[1];
                     }
                 }
@@ -423,17 +433,28 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     // issuer's bounded wait runs out and the CTA unwinds with WAIT_TIMEOUT
                     const bool withhold = b.withhold_test && blockIdx.x == 0 && u == unit0 && kb == 0;
                     if (!withhold) {
+                        if (x.rows_mode && g.g3d) {
+                            if (PAIR == 2) tma_load_3d_pair(sa, tm_rows, &full_bar[stage], 0, kb * BK, coord[0]);
+                            else tma_load_3d(sa, tm_rows, &full_bar[stage], 0, kb * BK, coord[0]);
+                        } else {
 #pragma unroll
-                        for (int s = 0; s < 4; ++s)
-                            if (coord[s] >= 0) {
-                                if (PAIR == 2) tma_load_2d_pair(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
-                                else tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
+                            for (int s = 0; s < 4; ++s)
+                                if (coord[s] >= 0) {
+                                    if (PAIR == 2) tma_load_2d_pair(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
+                                    else tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], coord[s], kb * BK);
+                                }
+                        }
+                        if (g.a3d) {                      // the CTA's column chunks in one load
+                            const int chunk = (x.nt * BN + (int)crank * B_COLS) / 64;
+                            if (PAIR == 2) tma_load_3d_pair(sb, &g.tm_a, &full_bar[stage], 0, kb * BK, chunk);
+                            else tma_load_3d(sb, &g.tm_a, &full_bar[stage], 0, kb * BK, chunk);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < B_COLS / 64; ++j) {
+                                const int col = x.nt * BN + (int)crank * B_COLS + j * 64;
+                                if (PAIR == 2) tma_load_2d_pair(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], col, kb * BK);
+                                else tma_load_2d(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], col, kb * BK);
                             }
-#pragma unroll
-                        for (int j = 0; j < B_COLS / 64; ++j) {
-                            const int col = x.nt * BN + (int)crank * B_COLS + j * 64;
-                            if (PAIR == 2) tma_load_2d_pair(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], col, kb * BK);
-                            else tma_load_2d(sb + j * B_BOX_BYTES, &g.tm_a, &full_bar[stage], col, kb * BK);
                         }
                     }
                     issued[stage] = true;
@@ -625,6 +646,22 @@ bool encode_bf16(CUtensorMap *m, const void *base, int width, int T, int64_t ld,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 3-D map over a token-major matrix [T x ld] seen as {inner, T, chunks}: element
+// (i, t, k) is base[t * ld + k * inner + i]; box {inner, 64, box_chunks}.
+bool encode_bf16_chunks(CUtensorMap *m, const void *base, int inner, int T, int chunks, int64_t ld,
+                        int box_chunks, CUtensorMapSwizzle sw)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)(T > 0 ? T : 1), (cuuint64_t)chunks};
+    const cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)inner * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)inner, (cuuint32_t)BK, (cuuint32_t)box_chunks};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Groups of a call: runs of consecutive problems with the same A, stride, C and T.
 struct HostGroup {
     int first, count;
@@ -810,7 +847,10 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
             const sf_dw_problem &p0 = probs[hg.first];
             DwGroup &g = gd[k - gi];
             const void *a = p0.T > 0 ? p0.A : p0.dW;     // any valid address when there are no tokens
-            if (!encode_bf16(&g.tm_a, a, p0.C, p0.T, p0.T > 0 ? p0.ld_a : p0.C, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+            const int64_t lda = p0.T > 0 ? p0.ld_a : p0.C;
+            g.a3d = p0.C % 64 == 0 &&
+                    encode_bf16_chunks(&g.tm_a, a, 64, p0.T, p0.C / 64, lda, B_COLS / 64, CU_TENSOR_MAP_SWIZZLE_128B);
+            if (!g.a3d && !encode_bf16(&g.tm_a, a, p0.C, p0.T, lda, 64, CU_TENSOR_MAP_SWIZZLE_128B))
                 rc = SF_ERR_CUDA;
             g.first = pi;
             g.count = hg.count;
@@ -823,7 +863,8 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
                 g.info = reinterpret_cast<const int32_t *>(base);
                 g.rowmap = reinterpret_cast<const int32_t *>(base + kInfoBytes);
                 const void *dxg = base + kInfoBytes + rowmap_bytes(hg.mcap);
-                if (!encode_bf16(&g.tm_g, dxg, hg.mcap, p0.T, hg.mcap, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+                g.g3d = encode_bf16_chunks(&g.tm_g, dxg, 32, p0.T, hg.mcap / 32, hg.mcap, 4, CU_TENSOR_MAP_SWIZZLE_64B);
+                if (!g.g3d && !encode_bf16(&g.tm_g, dxg, hg.mcap, p0.T, hg.mcap, 32, CU_TENSOR_MAP_SWIZZLE_64B))
                     rc = SF_ERR_CUDA;
             }
             long long tiles_mt = 0;
