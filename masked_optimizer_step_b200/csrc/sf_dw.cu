@@ -110,12 +110,13 @@ struct alignas(64) DwGroup {
     // B_COLS / 64}: one load brings the CTA's column chunks of a stage, chunk after chunk (the
     // layout the four 2-D boxes give); otherwise 2-D {C, T}, box {64, 64}. 128-byte swizzle.
     CUtensorMap tm_a;
-    // gathered rows: 3-D {32 rows, T, mcap / 32 chunks}, box {32, 64, 4}, 64-byte swizzle (or
-    // 2-D {mcap, T}, box {32, 64}, when the 3-D map is not accepted)
+    // gathered rows, stored row by row (each row's tokens contiguous, stride tp): 2-D {T, mcap},
+    // box {64 tokens, 128 rows}, 128-byte swizzle -- a K-major operand, as the tensor cores read
+    // fastest; tokens from T to tp are outside the map and read as zeros
     CUtensorMap tm_g;
     const int32_t *info;         // device: [0] mode (1 = rows), [1] gathered rows (null: tiles only)
     const int32_t *rowmap;       // device: per gathered row, (slot << 3) | problem, or -1
-    int32_t first, count, C, T, n_ntiles, mcap, a3d, g3d;   // g3d: tm_g is 3-D (else 2-D, box {32, 64})
+    int32_t first, count, C, T, n_ntiles, mcap, a3d;
 };
 
 struct DwBatch {
@@ -137,10 +138,10 @@ struct GatherProb {
 };
 
 struct GatherGroup {
-    uint16_t *dxg;
+    uint16_t *dxg;               // [mcap x tp]: gathered row k holds dX[t, r_k] at dxg[k * tp + t]
     int32_t *info;
     int32_t *rowmap;
-    int32_t first, count, T, mcap;
+    int32_t first, count, T, mcap, tp;
 };
 
 constexpr int kMaxGatherGroups = 192;
@@ -175,9 +176,20 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 constexpr uint32_t kLayoutSW128 = 2;
 constexpr uint32_t kLayoutSW64 = 4;
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both MN-major, N, M.
+// Instruction descriptors, kind::f16: fp32 accumulator, bf16 A and B, N, M. Tile mode reads dX
+// in place, so both operands are MN-major (bits 15, 16); row mode's gathered rows are K-major.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                             ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(UM >> 4) << 24);
+constexpr uint32_t kIdescRows = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                                ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(UM >> 4) << 24);
+
+// K-major, 128-byte swizzle: rows of 128 bytes (64 tokens), 8-row groups 1024 bytes apart; the
+// leading offset is unused for this layout.
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t addr)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           (1ull << 46) | ((uint64_t)2u << 61);
+}
 
 // Row mode when the group's active rows fit the scratch and need fewer units than the mask
 // tiles do. Every reader computes the same answer from the same counts.
@@ -187,8 +199,8 @@ __device__ __forceinline__ bool choose_rows(int rows, int tiles_mt, int mcap)
 }
 
 // ------------------------------------ gather kernel ------------------------------------
-// Row mode: dxg[t, k] = dX_p[t, r] for the group's k-th active row r (problems in call order,
-// rows ascending), and rowmap[k] = (slot(r) << 3) | p. One CTA per (group, 32 tokens); a thread
+// Row mode: dxg[k, t] = dX_p[t, r] for the group's k-th active row r (problems in call order,
+// rows ascending; each gathered row's tokens contiguous), and rowmap[k] = (slot(r) << 3) | p. One CTA per (group, 32 tokens); a thread
 // takes a gathered row and issues its 32 token loads back to back. The reads are single
 // elements spread over dX: each one costs the DRAM fetch of the line around it, so in a group
 // with fewer than one active row in 16 the loads ask L2 for 64-byte fetches instead of the
@@ -196,8 +208,8 @@ __device__ __forceinline__ bool choose_rows(int rows, int tiles_mt, int mcap)
 // gathered element, the pass ~30% faster); denser groups use whole lines, which they need
 // anyway (64-byte fetches measured ~3x slower at 50%). Many small independent loads per thread
 // keep enough requests in flight.
-// Consecutive threads take consecutive gathered rows, so the writes coalesce. The first CTA of
-// a group records the mode and the row map, which the main kernel (next on the stream) reads.
+// A thread writes its row's 32 tokens as 64 contiguous bytes. The first CTA of a group records
+// the mode and the row map, which the main kernel (next on the stream) reads.
 __global__ void __launch_bounds__(kGatherThreads)
 dw_gather_kernel(const __grid_constant__ GatherBatch b, int blocks_per_group)
 {
@@ -240,7 +252,7 @@ dw_gather_kernel(const __grid_constant__ GatherBatch b, int blocks_per_group)
         }
         if (nt <= 0) continue;
         const uint16_t *src = p.dx + (size_t)t0 * p.ld_dx + r;
-        uint16_t *dst = g.dxg + (size_t)t0 * g.mcap + k;
+        uint16_t *dst = g.dxg + (size_t)k * g.tp + t0;
         uint16_t v[kGatherTokens];
         if (s_sparse) {
 #pragma unroll
@@ -251,9 +263,19 @@ dw_gather_kernel(const __grid_constant__ GatherBatch b, int blocks_per_group)
             for (int t = 0; t < kGatherTokens; ++t)
                 if (t < nt) v[t] = __ldcs(src + (size_t)t * p.ld_dx);
         }
+        if (nt == kGatherTokens) {            // t0 is a multiple of 32 and tp of 8: 16-byte aligned
 #pragma unroll
-        for (int t = 0; t < kGatherTokens; ++t)
-            if (t < nt) dst[(size_t)t * g.mcap] = v[t];
+            for (int q4 = 0; q4 < kGatherTokens / 8; ++q4) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w[e] = (uint32_t)v[8 * q4 + 2 * e] | ((uint32_t)v[8 * q4 + 2 * e + 1] << 16);
+                *reinterpret_cast<uint4 *>(dst + 8 * q4) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        } else {
+#pragma unroll
+            for (int t = 0; t < kGatherTokens; ++t)
+                if (t < nt) dst[t] = v[t];
+        }
     }
 }
 
@@ -388,20 +410,11 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 const CUtensorMap *tm_rows;
                 int coord[4];
                 int nvalid = 0;
-                if (x.rows_mode && g.g3d) {         // one 3-D box: the CTA's four 32-row chunks
+                if (x.rows_mode) {                  // one K-major box: the CTA's 128 gathered rows
                     tm_rows = &g.tm_g;
-                    coord[0] = (x.mt * UM + (int)crank * BM) / 32;
+                    coord[0] = x.mt * UM + (int)crank * BM;
                     coord[1] = coord[2] = coord[3] = -1;
                     nvalid = 4;
-                } else if (x.rows_mode) {
-                    tm_rows = &g.tm_g;
-                    const int total = g.info[1];
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        const int k0 = x.mt * UM + (int)crank * BM + s * 32;
-                        coord[s] = k0 < total ? k0 : -1;
-                        nvalid += coord[s] >= 0;
-                    }
                 } else {
                     const DwProb &p = prb(b, x.p);
                     tm_rows = &p.tm_dx;
@@ -419,7 +432,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 if (PAIR == 2 && leader) {
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
-                        if (x.rows_mode) nvalid_peer += g.g3d || x.mt * UM + BM + s * 32 < g.info[1];
+                        if (x.rows_mode) nvalid_peer += 1;
                         else nvalid_peer += x.mt * UNIT_TILES + 4 + s < prb(b, x.p).counts[1];
                     }
                 }
@@ -433,9 +446,9 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     // issuer's bounded wait runs out and the CTA unwinds with WAIT_TIMEOUT
                     const bool withhold = b.withhold_test && blockIdx.x == 0 && u == unit0 && kb == 0;
                     if (!withhold) {
-                        if (x.rows_mode && g.g3d) {
-                            if (PAIR == 2) tma_load_3d_pair(sa, tm_rows, &full_bar[stage], 0, kb * BK, coord[0]);
-                            else tma_load_3d(sa, tm_rows, &full_bar[stage], 0, kb * BK, coord[0]);
+                        if (x.rows_mode) {
+                            if (PAIR == 2) tma_load_2d_pair(sa, tm_rows, &full_bar[stage], kb * BK, coord[0]);
+                            else tma_load_2d(sa, tm_rows, &full_bar[stage], kb * BK, coord[0]);
                         } else {
 #pragma unroll
                             for (int s = 0; s < 4; ++s)
@@ -491,6 +504,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
             for (int u = unit0; u < total_units && ok; u += ustep) {
                 const Unit x = decode(u, sp, b);
                 const int nk = (grp(b, x.g).T + BK - 1) / BK;
+                const uint32_t idesc = x.rows_mode ? kIdescRows : kIdesc;
                 for (int kb = 0; kb < nk; ++kb) {
                     const int in_chunk = kb % CHUNK_STAGES;
                     if (in_chunk == 0) {             // a fresh chunk: wait until its buffer is drained
@@ -504,11 +518,14 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
 #pragma unroll
                     for (int k = 0; k < BK / UMMA_K; ++k) {
-                        // 16 tokens = 16 rows of 64 B (A-operand) or 128 B (B-operand)
-                        const uint64_t da = smem_desc(sa + k * UMMA_K * 64, A_TILE_BYTES, 8 * 64, kLayoutSW64);
+                        // 16 tokens: 32 bytes into each K-major row (row mode), or 16 rows of 64 B
+                        // (tile mode's A-operand) and of 128 B (the B-operand)
+                        const uint64_t da = x.rows_mode
+                            ? kmajor_sw128_desc(sa + k * UMMA_K * 2)
+                            : smem_desc(sa + k * UMMA_K * 64, A_TILE_BYTES, 8 * 64, kLayoutSW64);
                         const uint64_t db = smem_desc(sb + k * UMMA_K * 128, B_BOX_BYTES, 8 * 128, kLayoutSW128);
-                        if (PAIR == 2) mma_bf16_pair(d_tmem, da, db, kIdesc, (in_chunk | k) != 0);
-                        else mma_bf16(d_tmem, da, db, kIdesc, (in_chunk | k) != 0);
+                        if (PAIR == 2) mma_bf16_pair(d_tmem, da, db, idesc, (in_chunk | k) != 0);
+                        else mma_bf16(d_tmem, da, db, idesc, (in_chunk | k) != 0);
                     }
                     if (PAIR == 2) mma_commit_pair(&empty_bar[stage], 3);   // both CTAs' stages free
                     else mma_commit(&empty_bar[stage]);
@@ -662,6 +679,21 @@ bool encode_bf16_chunks(CUtensorMap *m, const void *base, int inner, int T, int 
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 2-D map over the gathered rows [mcap x tp] (row k's tokens contiguous), valid tokens T:
+// box {64 tokens, 128 rows}, 128-byte swizzle (a K-major operand tile).
+bool encode_rows_kmajor(CUtensorMap *m, const void *base, int T, int mcap, int64_t tp)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)mcap};
+    const cuuint64_t strides[1] = {(cuuint64_t)tp * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Groups of a call: runs of consecutive problems with the same A, stride, C and T.
 struct HostGroup {
     int first, count;
@@ -692,7 +724,7 @@ int plan_groups(const sf_dw_problem *probs, int n, HostGroup *out, size_t *ws_to
         g.mcap = (int)round_up(cap, 32);
         g.ws_off = off;
         off += kInfoBytes + rowmap_bytes(g.mcap) +
-               round_up((size_t)(probs[i].T > 0 ? probs[i].T : 0) * g.mcap * 2, 256);
+               round_up((size_t)round_up(probs[i].T > 0 ? probs[i].T : 0, 8) * g.mcap * 2, 256);
         i = j;
     }
     *ws_total = off;
@@ -790,6 +822,7 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
             g.count = hg.count;
             g.T = probs[hg.first].T;
             g.mcap = hg.mcap;
+            g.tp = (int)round_up((size_t)g.T, 8);
             tok_blocks = max(tok_blocks, (g.T + kGatherTokens - 1) / kGatherTokens);
             for (int q = 0; q < hg.count; ++q) {
                 const sf_dw_problem &p = probs[hg.first + q];
@@ -863,8 +896,7 @@ extern "C" int sf_masked_dw_phase(const sf_dw_problem *probs, int n, void *ws, s
                 g.info = reinterpret_cast<const int32_t *>(base);
                 g.rowmap = reinterpret_cast<const int32_t *>(base + kInfoBytes);
                 const void *dxg = base + kInfoBytes + rowmap_bytes(hg.mcap);
-                g.g3d = encode_bf16_chunks(&g.tm_g, dxg, 32, p0.T, hg.mcap / 32, hg.mcap, 4, CU_TENSOR_MAP_SWIZZLE_64B);
-                if (!g.g3d && !encode_bf16(&g.tm_g, dxg, hg.mcap, p0.T, hg.mcap, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+                if (!encode_rows_kmajor(&g.tm_g, dxg, p0.T, hg.mcap, (int64_t)round_up((size_t)p0.T, 8)))
                     rc = SF_ERR_CUDA;
             }
             long long tiles_mt = 0;

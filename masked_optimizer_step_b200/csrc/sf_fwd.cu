@@ -34,13 +34,25 @@
 namespace sf {
 namespace {
 
-constexpr int FM = 128;                 // tokens per unit
+#ifndef SF_FWD_PAIR
+#define SF_FWD_PAIR 1
+#endif
+// CTAs sharing a unit: with 2, a cluster pair runs one tcgen05.mma with cta_group::2 (M = 256
+// tokens): each CTA loads its own 128 tokens of A and its own 128 of the unit's 256 weight rows
+// (completing on the even CTA's barriers), so each SM loads 32 KB per stage instead of 48 KB.
+// Measured on B200 (parity green in both builds), one 7B layer at 2,048 tokens: 1,248 vs 1,222
+// TFLOP/s; 32 layers: 1,020 vs 1,114. One CTA per unit is the default.
+constexpr int FPAIR = SF_FWD_PAIR;
+static_assert(FPAIR == 1 || FPAIR == 2, "one CTA or a CTA pair per unit");
+constexpr int FM = 128;                 // tokens per CTA (TMEM lanes)
+constexpr int FUM = FM * FPAIR;         // tokens per unit
 constexpr int FN = 256;                 // weight rows per unit
+constexpr int FNC = FN / FPAIR;         // weight rows each CTA loads
 constexpr int FK = 64;                  // columns of C per stage (128 bytes of bf16)
 constexpr int F_UMMA_K = 16;
-constexpr int F_STAGES = 4;
+constexpr int F_STAGES = FPAIR == 2 ? 6 : 4;
 constexpr int F_A_BYTES = FM * FK * 2;              // 16 KB
-constexpr int F_W_BYTES = FN * FK * 2;              // 32 KB
+constexpr int F_W_BYTES = FNC * FK * 2;             // 32 KB (16 KB per CTA of a pair)
 constexpr int F_STAGE_BYTES = F_A_BYTES + F_W_BYTES;
 constexpr int F_CHUNK_STAGES = 1024 / FK;           // accumulation chunk: 1024 columns of C
 constexpr int F_NBUF = 2;
@@ -53,7 +65,7 @@ constexpr int F_MAX_PROBS = 96;
 
 // kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, N, M.
 constexpr uint32_t kFwdIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(FN >> 3) << 17) |
-                               ((uint32_t)(FM >> 4) << 24);
+                               ((uint32_t)(FUM >> 4) << 24);
 constexpr uint32_t kSW128 = 2;
 
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr)
@@ -66,7 +78,7 @@ __device__ __forceinline__ uint64_t kmajor_desc(uint32_t addr)
 
 struct alignas(64) FwdProb {
     CUtensorMap tm_a;            // A: dims {C, T}, box {64, 128}, 128-byte swizzle
-    CUtensorMap tm_w;            // W: dims {C, R}, box {64, 256}, 128-byte swizzle
+    CUtensorMap tm_w;            // W: dims {C, R}, box {64, 256 / pair}, 128-byte swizzle
     uint16_t *Y;
     int64_t ld_y;
     uint32_t *accum;
@@ -112,6 +124,9 @@ __device__ __forceinline__ uint32_t tracked_magnitude(uint32_t bits, bool &nonfi
 __global__ void __launch_bounds__(F_THREADS, 1)
 forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
 {
+    const uint32_t crank = FPAIR == 2 ? cluster_ctarank() : 0u;
+    const bool leader = crank == 0;
+    const int unit0 = blockIdx.x / FPAIR, ustep = gridDim.x / FPAIR;
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t full_bar[F_STAGES], empty_bar[F_STAGES], tfull_bar[F_NBUF], tempty_bar[F_NBUF], drain_bar;
     __shared__ uint32_t tmem_base_s;
@@ -130,14 +145,18 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
         }
         for (int a = 0; a < F_NBUF; ++a) {
             mbar_init(&tfull_bar[a], 1);
-            mbar_init(&tempty_bar[a], F_EPI_WARPS);
+            mbar_init(&tempty_bar[a], F_EPI_WARPS * FPAIR);     // the leader's counts both CTAs
         }
         mbar_init(&drain_bar, 1);
         fence_mbarrier_init();
     }
-    if (warp == 1) tmem_alloc(&tmem_base_s, F_TMEM_COLS);
+    if (warp == 1) {
+        if (FPAIR == 2) tmem_alloc_pair(&tmem_base_s, F_TMEM_COLS);
+        else tmem_alloc(&tmem_base_s, F_TMEM_COLS);
+    }
     tc_fence_before();
     __syncthreads();
+    if (FPAIR == 2) cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_s;
 
@@ -153,16 +172,22 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
             bool issued[F_STAGES] = {};
             uint32_t issued_parity[F_STAGES] = {};
             bool ok = true;
-            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+            for (int u = unit0; u < total_units && ok; u += ustep) {
                 const FUnit x = fdecode(b, u);
                 const FwdProb &p = b.p[x.p];
                 const int nk = (p.C + FK - 1) / FK;
+                const int t0 = x.mt * FUM + (int)crank * FM, r0 = x.nt * FN + (int)crank * FNC;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1u, &abort_flag)) { ok = false; break; }
                     uint8_t *sa = smem + stage * F_STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full_bar[stage], F_STAGE_BYTES);
-                    tma_load_2d(sa, &p.tm_a, &full_bar[stage], kb * FK, x.mt * FM);
-                    tma_load_2d(sa + F_A_BYTES, &p.tm_w, &full_bar[stage], kb * FK, x.nt * FN);
+                    if (leader) mbar_arrive_expect_tx(&full_bar[stage], FPAIR * F_STAGE_BYTES);
+                    if (FPAIR == 2) {
+                        tma_load_2d_pair(sa, &p.tm_a, &full_bar[stage], kb * FK, t0);
+                        tma_load_2d_pair(sa + F_A_BYTES, &p.tm_w, &full_bar[stage], kb * FK, r0);
+                    } else {
+                        tma_load_2d(sa, &p.tm_a, &full_bar[stage], kb * FK, t0);
+                        tma_load_2d(sa + F_A_BYTES, &p.tm_w, &full_bar[stage], kb * FK, r0);
+                    }
                     issued[stage] = true;
                     issued_parity[stage] = phase;
                     if (++stage == F_STAGES) { stage = 0; phase ^= 1u; }
@@ -172,7 +197,7 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
             }
-            if (!ok || abort_flag) {
+            if ((!ok || abort_flag) && leader) {
                 for (int s = 0; s < F_STAGES; ++s) {
                     if (!issued[s]) continue;
                     const uint64_t t0 = globaltimer_ns();
@@ -182,13 +207,13 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
         }
     } else if (warp == 1) {
         // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             int stage = 0;
             uint32_t phase = 0;
             int buf = 0;
             uint32_t buf_phase = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+            for (int u = unit0; u < total_units && ok; u += ustep) {
                 const FUnit x = fdecode(b, u);
                 const int nk = (b.p[x.p].C + FK - 1) / FK;
                 for (int kb = 0; kb < nk; ++kb) {
@@ -203,18 +228,26 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
                     const uint32_t sw = sa + F_A_BYTES;
                     const uint32_t d_tmem = tmem_base + (uint32_t)(buf * FN);
 #pragma unroll
-                    for (int k = 0; k < FK / F_UMMA_K; ++k)       // 16 columns of C = 32 bytes
-                        mma_bf16(d_tmem, kmajor_desc(sa + k * 32), kmajor_desc(sw + k * 32), kFwdIdesc,
-                                 (in_chunk | k) != 0);
-                    mma_commit(&empty_bar[stage]);
+                    for (int k = 0; k < FK / F_UMMA_K; ++k) {     // 16 columns of C = 32 bytes
+                        if (FPAIR == 2)
+                            mma_bf16_pair(d_tmem, kmajor_desc(sa + k * 32), kmajor_desc(sw + k * 32), kFwdIdesc,
+                                          (in_chunk | k) != 0);
+                        else
+                            mma_bf16(d_tmem, kmajor_desc(sa + k * 32), kmajor_desc(sw + k * 32), kFwdIdesc,
+                                     (in_chunk | k) != 0);
+                    }
+                    if (FPAIR == 2) mma_commit_pair(&empty_bar[stage], 3);
+                    else mma_commit(&empty_bar[stage]);
                     if (++stage == F_STAGES) { stage = 0; phase ^= 1u; }
                     if (in_chunk == F_CHUNK_STAGES - 1 || kb == nk - 1) {
-                        mma_commit(&tfull_bar[buf]);
+                        if (FPAIR == 2) mma_commit_pair(&tfull_bar[buf], 3);
+                        else mma_commit(&tfull_bar[buf]);
                         if (++buf == F_NBUF) { buf = 0; buf_phase ^= 1u; }
                     }
                 }
             }
-            mma_commit(&drain_bar);
+            if (FPAIR == 2) mma_commit_pair(&drain_bar, 3);
+            else mma_commit(&drain_bar);
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&drain_bar, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {}
         }
@@ -226,11 +259,11 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
         int buf = 0;
         uint32_t buf_phase = 0;
         bool nonfinite = false;
-        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+        for (int u = unit0; u < total_units; u += ustep) {
             const FUnit x = fdecode(b, u);
             const FwdProb &p = b.p[x.p];
             const int nk = (p.C + FK - 1) / FK;
-            const int t = x.mt * FM + quad * 32 + lane;             // this lane's token
+            const int t = x.mt * FUM + (int)crank * FM + quad * 32 + lane;   // this lane's token
             const int r0 = x.nt * FN + half * F_EPI_COLS;           // first weight row of the half
             float acc[F_EPI_COLS];
 #pragma unroll
@@ -252,7 +285,10 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+                if (lane == 0) {
+                    if (FPAIR == 2 && !leader) mbar_arrive_remote(&tempty_bar[buf], 0);
+                    else mbar_arrive(&tempty_bar[buf]);
+                }
                 if (++buf == F_NBUF) { buf = 0; buf_phase ^= 1u; }
             }
             if (!ready) break;
@@ -292,10 +328,12 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    if (FPAIR == 2) cluster_sync();            // neither CTA leaves while the pair's MMAs may run
     if (abort_flag && tid == 0) set_status(status, SF_STATUS_WAIT_TIMEOUT);
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, F_TMEM_COLS);
+        if (FPAIR == 2) tmem_dealloc_pair(tmem_base, F_TMEM_COLS);
+        else tmem_dealloc(tmem_base, F_TMEM_COLS);
     }
 }
 
@@ -356,6 +394,22 @@ extern "C" int sf_forward_tracked(const sf_fwd_problem *probs, int n, uint32_t *
     if (cudaFuncSetAttribute(forward_tracked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)F_SMEM_BYTES) != cudaSuccess)
         return SF_ERR_CUDA;
+    int pair_slots = 0;                       // CTA pairs that can be resident at once
+    if (FPAIR == 2) {
+        cudaLaunchConfig_t qcfg = {};
+        cudaLaunchAttribute qattr;
+        qattr.id = cudaLaunchAttributeClusterDimension;
+        qattr.val.clusterDim.x = 2;
+        qattr.val.clusterDim.y = 1;
+        qattr.val.clusterDim.z = 1;
+        qcfg.gridDim = dim3(2 * sms);
+        qcfg.blockDim = dim3(F_THREADS);
+        qcfg.dynamicSmemBytes = F_SMEM_BYTES;
+        qcfg.attrs = &qattr;
+        qcfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&pair_slots, forward_tracked_kernel, &qcfg) != cudaSuccess || pair_slots <= 0)
+            return SF_ERR_CUDA;
+    }
     cudaStream_t st = as_stream(stream);
     FwdBatch *batch = new FwdBatch;
     int rc = SF_OK;
@@ -368,7 +422,7 @@ extern "C" int sf_forward_tracked(const sf_fwd_problem *probs, int n, uint32_t *
             FwdProb &d = batch->p[batch->n_prob];
             if (p.T == 0) continue;                       // no tokens: nothing to compute or fold
             if (!encode_kmajor(&d.tm_a, p.A, p.C, p.T, p.ld_a, FM) ||
-                !encode_kmajor(&d.tm_w, p.W, p.C, p.mask.R, p.ld_w, FN)) {
+                !encode_kmajor(&d.tm_w, p.W, p.C, p.mask.R, p.ld_w, FNC)) {
                 rc = SF_ERR_CUDA;
                 break;
             }
@@ -378,7 +432,7 @@ extern "C" int sf_forward_tracked(const sf_fwd_problem *probs, int n, uint32_t *
             d.T = p.T;
             d.C = p.C;
             d.R = p.mask.R;
-            d.n_mt = (p.T + FM - 1) / FM;
+            d.n_mt = (p.T + FUM - 1) / FUM;
             d.n_nt = (p.mask.R + FN - 1) / FN;
             d.unit_begin = units;
             units += d.n_mt * d.n_nt;
@@ -386,9 +440,23 @@ extern "C" int sf_forward_tracked(const sf_fwd_problem *probs, int n, uint32_t *
         }
         if (rc != SF_OK || batch->n_prob == 0) continue;
         batch->total_units = units;
-        const int grid = units < sms ? units : sms;
-        forward_tracked_kernel<<<grid, F_THREADS, F_SMEM_BYTES, st>>>(*batch, dev_status);
-        if (launch_status() != SF_OK) rc = SF_ERR_CUDA;
+        const int slots = FPAIR == 2 ? pair_slots : sms;
+        const int grid = FPAIR * (units < slots ? units : slots);
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(F_THREADS);
+        cfg.dynamicSmemBytes = F_SMEM_BYTES;
+        cfg.stream = st;
+        cfg.attrs = &attr;
+        cfg.numAttrs = FPAIR == 2 ? 1 : 0;
+        if (cudaLaunchKernelEx(&cfg, forward_tracked_kernel, *batch, dev_status) != cudaSuccess ||
+            launch_status() != SF_OK)
+            rc = SF_ERR_CUDA;
     }
     delete batch;
     return rc;
