@@ -205,7 +205,7 @@ int sf_embed_grad(const int32_t *tokens, int n_tok, const void *dY, int H, int64
  * latency-critical loop that cannot afford cudaMalloc's implicit synchronisation). The scratch
  * is a fixed array of SF_EMBED_NOALLOC_SCRATCH_INTS int32 (256 KiB) in the library's own device
  * memory, present on every GPU that loads the library until the process exits; a call needs
- * slot_cap + 1 + n_tok of them and returns SF_ERR_UNSUPPORTED beyond that. The first call on a
+ * 4 * slot_cap + 4 + n_tok of them and returns SF_ERR_UNSUPPORTED beyond that. The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) and caches it for the
  * device's current context (a new context, e.g. after cudaDeviceReset, repeats the lookup); make
  * that first call before any stream capture. All calls on a GPU share the array: calls that can

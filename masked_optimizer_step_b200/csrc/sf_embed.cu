@@ -7,14 +7,17 @@
 // conductor marks active are computed and stored.
 //
 // Two launches:
-//   embed_index_kernel  one CTA: for every token whose row is active, its slot; per-slot counts
-//                       (shared-memory atomics, exact), an exclusive scan into segment offsets,
-//                       and a stable scatter of token positions into their slot's segment of ws
-//                       (ascending within a segment, so the sum order is fixed).
-//   embed_sum_kernel    persistent: one item = (active row, 256-column chunk). 8 warps each
-//                       sum every 8th token of the row's sorted segment with 16-byte loads (eight
-//                       in flight per lane) and the partial sums are added in warp order. Active
-//                       rows without tokens get zeros.
+//   embed_index_kernel  one CTA: for every token whose row is active, its slot (the loads of four
+//                       tokens per thread in flight together, the slots kept in shared memory);
+//                       per-slot counts (shared-memory atomics, exact), an exclusive scan into
+//                       segment offsets, a table of (slot, segment) per active row, a scatter of
+//                       the token positions into their slot's segment, and a sort of each segment
+//                       (one warp per segment, through a bitmap of positions) so that positions
+//                       are ascending within a segment and the sum order is fixed.
+//   embed_sum_kernel    persistent: one item = (table entry, 256-column chunk). 8 warps each sum
+//                       every 8th token of the row's sorted segment with 16-byte loads (up to
+//                       eight in flight per lane) and the partial sums are added in warp order.
+//                       Active rows without tokens get zeros.
 // Traffic: dY rows of the tokens of active rows are read once per column chunk (8 KB per token
 // at H = 4096); 16 KB per active row is written.
 #include <atomic>
@@ -34,72 +37,172 @@ constexpr int kSumWarps = kSumThreads / 32;
 constexpr int kChunkCols = 256;             // 32 lanes x 8 bf16
 constexpr int kMaxTokens = 16384;
 constexpr int kMaxSlots = 49152;
-constexpr int kSumUnroll = 8;               // token loads in flight per lane
 
-// ws layout: seg_off[slot_cap + 1] int32 | perm[n_tok] int32
-__global__ void __launch_bounds__(kIndexThreads)
-embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int32_t *seg_off, int32_t *perm,
-                   uint32_t *status)
+// Scratch layout (int32 words): tbl[4 * slot_cap] | n_tbl[4] | perm[n_tok]
+//   tbl[j] = {slot, first, end, 0} of the j-th active row that holds a slot (active-row order);
+//   perm[first .. end) are that row's token positions, ascending.
+constexpr size_t scratch_ints(int n_tok, int slot_cap)
 {
-    extern __shared__ int cnt[];            // [slot_cap]
+    return 4 * (size_t)slot_cap + 4 + (size_t)n_tok;
+}
+
+constexpr int kBatch = 4;                   // tokens per thread whose loads are in flight together
+constexpr size_t kSmemLimit = 200 * 1024;   // dynamic shared memory of the index kernel, at most
+
+// Shared memory of the index kernel, in int32 words: cnt[slot_cap] | s_slot[n_tok] while the
+// slots are counted and scattered (s_slot only when it fits); afterwards the same space holds one
+// bitmap of n_tok bits per warp for the per-segment sort.
+constexpr size_t index_smem_ints(int n_tok, int slot_cap, bool keep_slots)
+{
+    const size_t a = (size_t)slot_cap + (keep_slots ? (size_t)n_tok : 0);
+    const size_t bm = (size_t)(kIndexThreads / 32) * (((size_t)n_tok + 31) / 32);
+    return a > bm ? a : bm;
+}
+
+// The slot of token id r, or -1 (bad id, inactive row, or a row without a slot). The mask word
+// and the slot are loaded together: both depend only on r.
+__device__ __forceinline__ int slot_of(int r, uint32_t word, int slot)
+{
+    return ((word >> (r & 31)) & 1u) ? slot : -1;
+}
+
+__device__ __forceinline__ int active_slot(const int32_t *tok, int t, const sf_mask &mk)
+{
+    const int r = tok[t];
+    if (r < 0 || r >= mk.R) return -1;
+    return slot_of(r, mk.words[r >> 5], mk.row_slot[r]);
+}
+
+__global__ void __launch_bounds__(kIndexThreads)
+embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int4 *tbl, int32_t *n_tbl, int32_t *perm,
+                   int keep_slots, uint32_t *status)
+{
+    extern __shared__ int smem_i[];
+    int *cnt = smem_i;
+    int *s_slot = smem_i + mk.slot_cap;
     __shared__ int scan_scratch[33];
-    __shared__ int s_run;
     const int cap = mk.slot_cap;
-    for (int s = threadIdx.x; s < cap; s += blockDim.x) cnt[s] = 0;
-    if (threadIdx.x == 0) s_run = 0;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_launch_dependents();                 // the sum kernel may start; it waits for this grid
+    for (int s = tid; s < cap; s += blockDim.x) cnt[s] = 0;
+    // the first blockDim active rows and their slots, for the table: loaded beside the first
+    // tokens' loads (row ids and count with the token ids, slots with the mask words)
+    const int n_act = mk.counts[0];
+    const int act_row0 = tid < mk.R ? mk.active_rows[tid] : -1;
+    int act_slot0 = -1;
     __syncthreads();
+    // 1. the slot of each token, kBatch tokens per thread at a time so that their loads overlap
+    //    (id, then mask word and slot together); exact counts
     bool bad = false;
-    for (int t = threadIdx.x; t < n_tok; t += blockDim.x) {
-        const int r = tok[t];
-        if (r < 0 || r >= mk.R) { bad = true; continue; }
-        if (!((mk.words[r >> 5] >> (r & 31)) & 1u)) continue;   // inactive row: dropped
-        const int s = mk.row_slot[r];
-        if (s >= 0) atomicAdd(&cnt[s], 1);
+    for (int base = 0; base < n_tok; base += kBatch * blockDim.x) {
+        int r[kBatch], sl[kBatch];
+        uint32_t w[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int t = base + u * (int)blockDim.x + tid;
+            r[u] = t < n_tok ? tok[t] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int t = base + u * (int)blockDim.x + tid;
+            const bool valid = r[u] >= 0 && r[u] < mk.R;
+            if (t < n_tok && !valid) bad = true;
+            w[u] = valid ? mk.words[r[u] >> 5] : 0u;
+            sl[u] = valid ? mk.row_slot[r[u]] : -1;
+        }
+        if (base == 0 && tid < n_act) act_slot0 = mk.row_slot[act_row0];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int t = base + u * (int)blockDim.x + tid;
+            sl[u] = r[u] >= 0 && r[u] < mk.R ? slot_of(r[u], w[u], sl[u]) : -1;
+            if (sl[u] >= 0) atomicAdd(&cnt[sl[u]], 1);
+            if (keep_slots && t < n_tok) s_slot[t] = sl[u];
+        }
     }
+    if (n_tok == 0 && tid < n_act) act_slot0 = mk.row_slot[act_row0];
     if (bad) set_status(status, SF_STATUS_BAD_TOKEN);
     __syncthreads();
-    // exclusive scan of the counts, in slot order, chunk by chunk
-    for (int base = 0; base < cap; base += blockDim.x) {
-        const int s = base + threadIdx.x;
-        const int c = s < cap ? cnt[s] : 0;
+    // 2. exclusive scan of the counts in slot order: each thread sums a run of consecutive slots,
+    //    one block scan over the runs; cnt[s] becomes segment s's start (and its fill cursor)
+    __shared__ int s_total;
+    {
+        const int per = (cap + (int)blockDim.x - 1) / (int)blockDim.x;
+        const int s0 = min(cap, tid * per), s1 = min(cap, s0 + per);
+        int local = 0;
+        for (int s = s0; s < s1; ++s) local += cnt[s];
         int total;
-        const int off = block_exclusive_scan(c, scan_scratch, &total);
-        const int run = s_run;
-        if (s < cap) {
-            seg_off[s] = run + off;
-            cnt[s] = 0;                     // becomes the fill cursor
+        int run = block_exclusive_scan(local, scan_scratch, &total);
+        for (int s = s0; s < s1; ++s) {
+            const int c = cnt[s];
+            cnt[s] = run;
+            run += c;
         }
-        __syncthreads();
-        if (threadIdx.x == 0) s_run = run + total;
-        __syncthreads();
+        if (tid == 0) s_total = total;
     }
-    if (threadIdx.x == 0) seg_off[cap] = s_run;
     __syncthreads();
-    // Stable scatter: a slot's positions land in ascending order. Tokens go in rounds of
-    // blockDim (one per thread, in order); inside a warp, lanes holding the same slot rank
-    // themselves by lane; across warps, each warp's group leaders claim their slots' next places
-    // in warp order, one warp per barrier step. So the sum order below never depends on timing.
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = (1u << lane) - 1u;
+    // 3. the table of active rows that hold a slot, in active-row order; a segment ends where
+    //    the next slot's begins
+    {
+        const int total = s_total;
+        int base_j = 0;
+        for (int base = 0; base < n_act; base += blockDim.x) {
+            const int k = base + tid;
+            const int sl = base == 0 ? act_slot0 : (k < n_act ? mk.row_slot[mk.active_rows[k]] : -1);
+            int tot;
+            const int j = block_exclusive_scan(sl >= 0, scan_scratch, &tot);
+            if (sl >= 0) tbl[base_j + j] = make_int4(sl, cnt[sl], sl + 1 < cap ? cnt[sl + 1] : total, 0);
+            base_j += tot;
+        }
+        if (tid == 0) n_tbl[0] = base_j;
+    }
+    __syncthreads();
+    // 4. every token of an active row into its slot's segment (in no particular order yet)
     for (int base = 0; base < n_tok; base += blockDim.x) {
-        const int t = base + threadIdx.x;
-        int s = -1;
-        if (t < n_tok) {
-            const int r = tok[t];
-            if (r >= 0 && r < mk.R && ((mk.words[r >> 5] >> (r & 31)) & 1u)) s = mk.row_slot[r];
-        }
-        const uint32_t peers = __match_any_sync(0xffffffffu, s);
-        const int leader = __ffs(peers) - 1;
-        int place = 0;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-            if (warp == w && s >= 0 && lane == leader) {
-                place = cnt[s];
-                cnt[s] = place + __popc(peers);
+        const int t = base + tid;
+        const int s = t < n_tok ? (keep_slots ? s_slot[t] : active_slot(tok, t, mk)) : -1;
+        if (s >= 0) perm[atomicAdd(&cnt[s], 1)] = t;
+    }
+    __syncthreads();
+    // 5. each segment sorted ascending, one warp per segment: its positions are set as bits of an
+    //    n_tok-bit map in shared memory and read back in bit order (a counting sort), so the
+    //    order the sums take below is fixed whatever order the atomics gave
+    {
+        const int words = (n_tok + 31) >> 5;
+        const int wpl = (words + 31) >> 5;             // bitmap words per lane
+        uint32_t *bm = reinterpret_cast<uint32_t *>(smem_i) + (size_t)warp * words;
+        const int n_seg = n_tbl[0];
+        for (int j = warp; j < n_seg; j += (int)(blockDim.x >> 5)) {
+            const int4 e = tbl[j];
+            const int first = e.y, m = e.z - e.y;
+            if (m < 2) continue;
+            for (int q = lane; q < words; q += 32) bm[q] = 0u;
+            __syncwarp();
+            for (int i0 = 0; i0 < m; i0 += 32 * kBatch * 2) {     // loads in flight, then the bits
+                int p[kBatch * 2];
+#pragma unroll
+                for (int u = 0; u < kBatch * 2; ++u) {
+                    const int i = i0 + u * 32 + lane;
+                    p[u] = i < m ? perm[first + i] : -1;
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch * 2; ++u)
+                    if (p[u] >= 0) atomicOr(&bm[p[u] >> 5], 1u << (p[u] & 31));
             }
-            __syncthreads();
+            __syncwarp();
+            const int q0 = min(words, lane * wpl), q1 = min(words, q0 + wpl);
+            int c = 0;
+            for (int q = q0; q < q1; ++q) c += __popc(bm[q]);
+            int out = first + warp_inclusive_scan(c) - c;
+            for (int q = q0; q < q1; ++q) {
+                uint32_t bits = bm[q];
+                while (bits) {
+                    const int b = __ffs(bits) - 1;
+                    perm[out++] = q * 32 + b;
+                    bits &= bits - 1u;
+                }
+            }
+            __syncwarp();
         }
-        place = __shfl_sync(0xffffffffu, place, leader);
-        if (s >= 0) perm[seg_off[s] + place + __popc(peers & lt)] = t;
     }
 }
 
@@ -113,77 +216,107 @@ __device__ __forceinline__ void add_bf16x8(float (&acc)[8], const uint4 &v)
     }
 }
 
-__global__ void __launch_bounds__(kSumThreads)
-embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, sf_mask mk, float *G, long long ld_g,
-                 const int32_t *seg_off, const int32_t *perm)
+// Adds the bf16 rows held by lanes j0 .. j0 + U - 1 of `mine` (token positions) into acc, in
+// that order, U loads in flight.
+template <int U>
+__device__ __forceinline__ void sum_batch(float (&acc)[8], const uint16_t *dY, long long ld_dy, int c0,
+                                          bool col_ok, int mine, int j0)
+{
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int p = __shfl_sync(0xffffffffu, mine, j0 + u);
+        if (col_ok) v[u] = __ldg(reinterpret_cast<const uint4 *>(dY + (size_t)p * ld_dy + c0));
+    }
+    if (col_ok) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) add_bf16x8(acc, v[u]);
+    }
+}
+
+__global__ void __launch_bounds__(kSumThreads, 2)
+embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, float *G, long long ld_g, const int4 *tbl,
+                 const int32_t *n_tbl, const int32_t *perm)
 {
     __shared__ float part[kSumWarps][kChunkCols];
-    const int n_act = mk.counts[0];
+    griddep_wait();                             // the index kernel's table and positions
     const int nchunks = (H + kChunkCols - 1) / kChunkCols;
-    const int total = n_act * nchunks;
+    const int total = n_tbl[0] * nchunks;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    int4 e_next = (int)blockIdx.x < total ? tbl[blockIdx.x / nchunks] : make_int4(0, 0, 0, 0);
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
-        const int k = item / nchunks;
-        const int chunk = item - k * nchunks;
-        const int r = mk.active_rows[k];
-        const int slot = mk.row_slot[r];
-        if (slot < 0) continue;
-        const int b0 = seg_off[slot], n = seg_off[slot + 1] - b0;
+        const int j = item / nchunks;
+        const int chunk = item - j * nchunks;
+        const int4 e = e_next;                  // slot, first, end
+        const int nxt = item + (int)gridDim.x;
+        if (nxt < total) e_next = tbl[nxt / nchunks];   // the next item's entry, loaded early
+        const int slot = e.x, b0 = e.y, n = e.z - e.y;
         const int c0 = chunk * kChunkCols + lane * 8;
         const bool col_ok = c0 < H;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         // warp w sums positions w, w + 8, w + 16, ... of the sorted segment, in that order; a
-        // batch holds the warp's next 32 positions, one per lane, handed out by shuffles
+        // batch holds the warp's next 32 positions, one per lane, handed out by shuffles and
+        // loaded 8, 4, 2, 1 at a time (the count is the same for the whole warp)
         for (int base = warp; base < n; base += kSumWarps * 32) {
             const int idx = base + kSumWarps * lane;
             const int mine = idx < n ? __ldg(perm + b0 + idx) : 0;
             const int cnt = min(32, (n - base + kSumWarps - 1) / kSumWarps);
-            for (int j0 = 0; j0 < cnt; j0 += kSumUnroll) {
-                uint4 v[kSumUnroll];
-#pragma unroll
-                for (int u = 0; u < kSumUnroll; ++u) {
-                    const int p = __shfl_sync(0xffffffffu, mine, (j0 + u) & 31);
-                    if (j0 + u < cnt && col_ok)
-                        v[u] = __ldg(reinterpret_cast<const uint4 *>(dY + (size_t)p * ld_dy + c0));
-                }
-#pragma unroll
-                for (int u = 0; u < kSumUnroll; ++u)
-                    if (j0 + u < cnt && col_ok) add_bf16x8(acc, v[u]);
-            }
+            int j0 = 0;
+            for (; j0 + 8 <= cnt; j0 += 8) sum_batch<8>(acc, dY, ld_dy, c0, col_ok, mine, j0);
+            if (cnt - j0 >= 4) { sum_batch<4>(acc, dY, ld_dy, c0, col_ok, mine, j0); j0 += 4; }
+            if (cnt - j0 >= 2) { sum_batch<2>(acc, dY, ld_dy, c0, col_ok, mine, j0); j0 += 2; }
+            if (cnt - j0 >= 1) sum_batch<1>(acc, dY, ld_dy, c0, col_ok, mine, j0);
         }
         // fixed-order combination of the 8 warps' partial sums
 #pragma unroll
-        for (int e = 0; e < 8; ++e) part[warp][lane * 8 + e] = acc[e];
+        for (int q = 0; q < 8; ++q) part[warp][lane * 8 + q] = acc[q];
         __syncthreads();
         const int col = chunk * kChunkCols + tid;
         if (col < H) {
-            float s = part[0][tid];
+            float sum = part[0][tid];
 #pragma unroll
-            for (int w = 1; w < kSumWarps; ++w) s = __fadd_rn(s, part[w][tid]);
-            G[(size_t)slot * ld_g + col] = s;
+            for (int w = 1; w < kSumWarps; ++w) sum = __fadd_rn(sum, part[w][tid]);
+            G[(size_t)slot * ld_g + col] = sum;
         }
         __syncthreads();
     }
 }
 
-// The two launches of one embedding-row gradient, on scratch seg_off[slot_cap + 1] | perm[n_tok].
+// The two launches of one embedding-row gradient, on scratch of scratch_ints(n_tok, slot_cap)
+// words (16-byte aligned).
 int launch_embed(const int32_t *tokens, int n_tok, const void *dY, int H, int64_t ld_dy, const sf_mask &mk,
                  float *G, int64_t ld_g, int32_t *scratch, uint32_t *dev_status, cudaStream_t st)
 {
-    int32_t *seg_off = scratch;
-    int32_t *perm = seg_off + mk.slot_cap + 1;
-    const size_t smem = (size_t)mk.slot_cap * sizeof(int);
+    int4 *tbl = reinterpret_cast<int4 *>(scratch);
+    int32_t *n_tbl = scratch + 4 * (size_t)mk.slot_cap;
+    int32_t *perm = n_tbl + 4;
+    const int keep_slots = index_smem_ints(n_tok, mk.slot_cap, true) * sizeof(int) <= kSmemLimit;
+    const size_t smem = index_smem_ints(n_tok, mk.slot_cap, keep_slots) * sizeof(int);
+    if (smem > kSmemLimit) return SF_ERR_UNSUPPORTED;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return SF_ERR_CUDA;
     const int sms = sm_count();
     if (sms <= 0) return SF_ERR_NO_DEVICE;
-    embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, mk, seg_off, perm, dev_status);
+    embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, mk, tbl, n_tbl, perm, keep_slots, dev_status);
     if (launch_status() != SF_OK) return SF_ERR_CUDA;
-    embed_sum_kernel<<<sms * 4, kSumThreads, 0, st>>>(static_cast<const uint16_t *>(dY), H, ld_dy,
-                                                      mk, G, ld_g, seg_off, perm);
+    // the sum kernel is launched as a programmatic dependent of the index kernel: its CTAs are
+    // placed while the index kernel runs and wait for its completion before reading the table
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sms * 4);
+    cfg.blockDim = dim3(kSumThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, embed_sum_kernel, static_cast<const uint16_t *>(dY), H, (long long)ld_dy, G,
+                           (long long)ld_g, static_cast<const int4 *>(tbl), static_cast<const int32_t *>(n_tbl),
+                           static_cast<const int32_t *>(perm)) != cudaSuccess)
+        return SF_ERR_CUDA;
     return launch_status();
 }
 
@@ -195,7 +328,7 @@ using namespace sf;
 extern "C" size_t sf_embed_grad_ws_bytes(int n_tok, int slot_cap)
 {
     if (n_tok < 0 || slot_cap < 0) return 0;
-    const size_t b = ((size_t)slot_cap + 1 + (size_t)n_tok) * sizeof(int32_t);
+    const size_t b = scratch_ints(n_tok, slot_cap) * sizeof(int32_t);
     return (b + 255) & ~(size_t)255;
 }
 
@@ -296,7 +429,7 @@ extern "C" int sf_embed_grad_noalloc(const int32_t *tokens, int n_tok, const voi
     int rc = check_mask(*mk);
     if (rc != SF_OK) return rc;
     if (n_tok > kMaxTokens || mk->slot_cap > kMaxSlots) return SF_ERR_UNSUPPORTED;
-    if ((long long)mk->slot_cap + 1 + n_tok > kNoAllocScratchInts) return SF_ERR_UNSUPPORTED;
+    if (scratch_ints(n_tok, mk->slot_cap) > (size_t)kNoAllocScratchInts) return SF_ERR_UNSUPPORTED;
     if ((H & 7) || ld_dy < H || (ld_dy & 7) || ld_g < H || (ld_g & 3)) return SF_ERR_ARG;
     if ((n_tok > 0 && !aligned16(dY)) || !aligned16(G)) return SF_ERR_ALIGN;
     if (mk->slot_cap == 0) return SF_OK;

@@ -60,13 +60,13 @@ def test_noalloc_matches_workspace_version_on_two_calls_in_a_row(sf):
 def test_noalloc_rejects_sizes_beyond_its_fixed_scratch(sf):
     lib = sf.load()
     V, n = 64, 16384
-    mk = sf.Mask(V, V, DEV)            # slot_cap + 1 + n_tok fits
+    mk = sf.Mask(V, V, DEV)            # 4 slot_cap + 4 + n_tok scratch ints fit
     sf.sf_mask_init(mk)
     dY = torch.zeros((n, 8), dtype=torch.bfloat16, device=DEV)
     tok = torch.zeros(n, dtype=torch.int32, device=DEV)
     G = torch.zeros((V, 8), device=DEV)
     sf.sf_embed_grad_noalloc(tok, dY, mk, G)
-    big = sf.Mask(49152, 49152, DEV)   # 49152 + 1 + 16384 > 65536 scratch ints: refused up front
+    big = sf.Mask(49152, 49152, DEV)   # 4 * 49152 + 4 + 16384 > 65536 scratch ints: refused up front
     m = big.struct()
     rc = lib.sf_embed_grad_noalloc(tok.data_ptr(), n, dY.data_ptr(), 8, 8, ctypes.byref(m),
                                    G.data_ptr(), 8, None, None)
