@@ -1112,7 +1112,7 @@ def main():
     hbm_kernel("update_kernel", stage_ms[3], upd_bytes, -(-len(plan0.upd_arr) // sf.SF_MATS_PER_LAUNCH),
                "24 B per active element (20 on fresh rows) + 8 B per row")
     if stage_ms[2] > 0:
-        kern["embed (index + sum)"] = {"ms_per_step": stage_ms[2] / K, "launches_per_step": 2,
+        kern["embed (index + sort + sum)"] = {"ms_per_step": stage_ms[2] / K, "launches_per_step": 3,
                                               "stream": "side (overlapped)" if not args.no_overlap_embedding else "main"}
     rated = [k for k, v in kern.items() if v.get("bound") in ("hbm", "tensor")]
     dominant = max(rated, key=lambda k: kern[k]["ms_per_step"])

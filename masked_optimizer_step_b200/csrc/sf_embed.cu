@@ -6,14 +6,14 @@
 // upstream gradients dY[t] over the batch positions t holding token r, and only rows the
 // conductor marks active are computed and stored.
 //
-// Two launches:
+// Three launches, each of the last two a programmatic dependent of the one before:
 //   embed_index_kernel  one CTA: for every token whose row is active, its slot (the loads of four
 //                       tokens per thread in flight together, the slots kept in shared memory);
 //                       per-slot counts (shared-memory atomics, exact), an exclusive scan into
-//                       segment offsets, a table of (slot, segment) per active row, a scatter of
-//                       the token positions into their slot's segment, and a sort of each segment
-//                       (one warp per segment, through a bitmap of positions) so that positions
-//                       are ascending within a segment and the sum order is fixed.
+//                       segment offsets, a table of (slot, segment) per active row, and a scatter
+//                       of the token positions into their slot's segment.
+//   embed_sort_kernel   one warp per segment over the whole grid: the segment's positions sorted
+//                       ascending through a bitmap of positions, so the sum order is fixed.
 //   embed_sum_kernel    persistent: one item = (table entry, 256-column chunk). 8 warps each sum
 //                       every 8th token of the row's sorted segment with 16-byte loads (up to
 //                       eight in flight per lane) and the partial sums are added in warp order.
@@ -48,16 +48,16 @@ constexpr size_t scratch_ints(int n_tok, int slot_cap)
 
 constexpr int kBatch = 4;                   // tokens per thread whose loads are in flight together
 constexpr size_t kSmemLimit = 200 * 1024;   // dynamic shared memory of the index kernel, at most
+constexpr int kIndexWarps = kIndexThreads / 32;
 
-// Shared memory of the index kernel, in int32 words: cnt[slot_cap] | s_slot[n_tok] while the
-// slots are counted and scattered (s_slot only when it fits); afterwards the same space holds one
-// bitmap of n_tok bits per warp for the per-segment sort.
+// The index kernel keeps the counts cnt[slot_cap] and, when they fit, each token's slot
+// s_slot[n_tok] in shared memory (otherwise the slots are looked up again for the scatter).
 constexpr size_t index_smem_ints(int n_tok, int slot_cap, bool keep_slots)
 {
-    const size_t a = (size_t)slot_cap + (keep_slots ? (size_t)n_tok : 0);
-    const size_t bm = (size_t)(kIndexThreads / 32) * (((size_t)n_tok + 31) / 32);
-    return a > bm ? a : bm;
+    return (size_t)slot_cap + (keep_slots ? (size_t)n_tok : 0);
 }
+
+constexpr int kSortThreads = 256;           // 8 warps, one segment at a time each
 
 // The slot of token id r, or -1 (bad id, inactive row, or a row without a slot). The mask word
 // and the slot are loaded together: both depend only on r.
@@ -73,17 +73,54 @@ __device__ __forceinline__ int active_slot(const int32_t *tok, int t, const sf_m
     return slot_of(r, mk.words[r >> 5], mk.row_slot[r]);
 }
 
+// One warp sorts the m >= 2 positions src[0 .. m) (a segment, in any order) into dst[0 .. m),
+// ascending (dst may be src): each position sets its bit in the warp's n_tok-bit map, and the set
+// bits are read back in order. Lane l owns the map words [l * wpl, (l + 1) * wpl): it alone
+// clears them and reads them back (a warp scan of the lanes' bit counts places its positions),
+// so only the bit setting needs the warp's barriers, and a next segment may start at once.
+__device__ __forceinline__ void sort_segment(const int32_t *src, int32_t *dst, int m, uint32_t *bm, int words,
+                                             int lane)
+{
+    const int wpl = (words + 31) >> 5;                       // bitmap words per lane
+    const int q0 = min(words, lane * wpl), q1 = min(words, q0 + wpl);
+    for (int q = q0; q < q1; ++q) bm[q] = 0u;
+    __syncwarp();
+    for (int i0 = 0; i0 < m; i0 += 32 * kBatch * 2) {        // loads in flight, then the bits
+        int p[kBatch * 2];
+#pragma unroll
+        for (int u = 0; u < kBatch * 2; ++u) {
+            const int i = i0 + u * 32 + lane;
+            p[u] = i < m ? src[i] : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch * 2; ++u)
+            if (p[u] >= 0) atomicOr(&bm[p[u] >> 5], 1u << (p[u] & 31));
+    }
+    __syncwarp();
+    int c = 0;
+    for (int q = q0; q < q1; ++q) c += __popc(bm[q]);
+    int out = warp_inclusive_scan(c) - c;
+    for (int q = q0; q < q1; ++q) {
+        uint32_t bits = bm[q];
+        while (bits) {
+            dst[out++] = q * 32 + __ffs(bits) - 1;
+            bits &= bits - 1u;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kIndexThreads)
 embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int4 *tbl, int32_t *n_tbl, int32_t *perm,
                    int keep_slots, uint32_t *status)
 {
     extern __shared__ int smem_i[];
-    int *cnt = smem_i;
-    int *s_slot = smem_i + mk.slot_cap;
-    __shared__ int scan_scratch[33];
     const int cap = mk.slot_cap;
+    int *cnt = smem_i;
+    int *s_slot = smem_i + cap;
+    __shared__ int scan_scratch[33];
+    __shared__ int s_total;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    griddep_launch_dependents();                 // the sum kernel may start; it waits for this grid
+    griddep_launch_dependents();                 // the sort kernel may start; it waits for this grid
     for (int s = tid; s < cap; s += blockDim.x) cnt[s] = 0;
     // the first blockDim active rows and their slots, for the table: loaded beside the first
     // tokens' loads (row ids and count with the token ids, slots with the mask words)
@@ -122,22 +159,33 @@ embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int4 *tbl, int32_t
     if (n_tok == 0 && tid < n_act) act_slot0 = mk.row_slot[act_row0];
     if (bad) set_status(status, SF_STATUS_BAD_TOKEN);
     __syncthreads();
-    // 2. exclusive scan of the counts in slot order: each thread sums a run of consecutive slots,
-    //    one block scan over the runs; cnt[s] becomes segment s's start (and its fill cursor)
-    __shared__ int s_total;
+    // 2. exclusive scan of the counts in slot order: warp w owns a contiguous run of slots, read
+    //    32 consecutive slots at a time (no bank conflicts); one scan over the warps' totals, then
+    //    each warp scans its run with a carry. cnt[s] becomes segment s's start (its fill cursor)
     {
-        const int per = (cap + (int)blockDim.x - 1) / (int)blockDim.x;
-        const int s0 = min(cap, tid * per), s1 = min(cap, s0 + per);
+        const int per_w = ((cap + kIndexWarps - 1) / kIndexWarps + 31) & ~31;
+        const int w0 = min(cap, warp * per_w), w1 = min(cap, w0 + per_w);
         int local = 0;
-        for (int s = s0; s < s1; ++s) local += cnt[s];
-        int total;
-        int run = block_exclusive_scan(local, scan_scratch, &total);
-        for (int s = s0; s < s1; ++s) {
-            const int c = cnt[s];
-            cnt[s] = run;
-            run += c;
+        for (int s = w0 + lane; s < w1; s += 32) local += cnt[s];
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) local += __shfl_xor_sync(0xffffffffu, local, d);
+        if (lane == 0) scan_scratch[warp] = local;
+        __syncthreads();
+        if (warp == 0) {
+            const int v = lane < kIndexWarps ? scan_scratch[lane] : 0;
+            const int inc = warp_inclusive_scan(v);
+            if (lane < kIndexWarps) scan_scratch[lane] = inc - v;
+            if (lane == 31) s_total = inc;
         }
-        if (tid == 0) s_total = total;
+        __syncthreads();
+        int carry = scan_scratch[warp];
+        for (int s0 = w0; s0 < w1; s0 += 32) {
+            const int s = s0 + lane;
+            const int c = s < w1 ? cnt[s] : 0;
+            const int inc = warp_inclusive_scan(c);
+            if (s < w1) cnt[s] = carry + inc - c;
+            carry += __shfl_sync(0xffffffffu, inc, 31);
+        }
     }
     __syncthreads();
     // 3. the table of active rows that hold a slot, in active-row order; a segment ends where
@@ -156,53 +204,32 @@ embed_index_kernel(const int32_t *tok, int n_tok, sf_mask mk, int4 *tbl, int32_t
         if (tid == 0) n_tbl[0] = base_j;
     }
     __syncthreads();
-    // 4. every token of an active row into its slot's segment (in no particular order yet)
+    // 4. every token of an active row into its slot's segment (in no particular order: the
+    //    sort kernel orders each segment)
     for (int base = 0; base < n_tok; base += blockDim.x) {
         const int t = base + tid;
         const int s = t < n_tok ? (keep_slots ? s_slot[t] : active_slot(tok, t, mk)) : -1;
         if (s >= 0) perm[atomicAdd(&cnt[s], 1)] = t;
     }
-    __syncthreads();
-    // 5. each segment sorted ascending, one warp per segment: its positions are set as bits of an
-    //    n_tok-bit map in shared memory and read back in bit order (a counting sort), so the
-    //    order the sums take below is fixed whatever order the atomics gave
-    {
-        const int words = (n_tok + 31) >> 5;
-        const int wpl = (words + 31) >> 5;             // bitmap words per lane
-        uint32_t *bm = reinterpret_cast<uint32_t *>(smem_i) + (size_t)warp * words;
-        const int n_seg = n_tbl[0];
-        for (int j = warp; j < n_seg; j += (int)(blockDim.x >> 5)) {
-            const int4 e = tbl[j];
-            const int first = e.y, m = e.z - e.y;
-            if (m < 2) continue;
-            for (int q = lane; q < words; q += 32) bm[q] = 0u;
-            __syncwarp();
-            for (int i0 = 0; i0 < m; i0 += 32 * kBatch * 2) {     // loads in flight, then the bits
-                int p[kBatch * 2];
-#pragma unroll
-                for (int u = 0; u < kBatch * 2; ++u) {
-                    const int i = i0 + u * 32 + lane;
-                    p[u] = i < m ? perm[first + i] : -1;
-                }
-#pragma unroll
-                for (int u = 0; u < kBatch * 2; ++u)
-                    if (p[u] >= 0) atomicOr(&bm[p[u] >> 5], 1u << (p[u] & 31));
-            }
-            __syncwarp();
-            const int q0 = min(words, lane * wpl), q1 = min(words, q0 + wpl);
-            int c = 0;
-            for (int q = q0; q < q1; ++q) c += __popc(bm[q]);
-            int out = first + warp_inclusive_scan(c) - c;
-            for (int q = q0; q < q1; ++q) {
-                uint32_t bits = bm[q];
-                while (bits) {
-                    const int b = __ffs(bits) - 1;
-                    perm[out++] = q * 32 + b;
-                    bits &= bits - 1u;
-                }
-            }
-            __syncwarp();
-        }
+}
+
+// Each segment of the table sorted ascending in place, one warp per segment over the whole
+// grid, so the order the sums take below is fixed whatever order the scatter's atomics gave.
+__global__ void __launch_bounds__(kSortThreads)
+embed_sort_kernel(const int4 *tbl, const int32_t *n_tbl, int32_t *perm, int n_tok)
+{
+    extern __shared__ uint32_t sort_bm[];        // one n_tok-bit map per warp
+    griddep_launch_dependents();                 // the sum kernel may start; it waits for this grid
+    griddep_wait();                              // the index kernel's table and scatter
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int words = (n_tok + 31) >> 5;
+    uint32_t *bm = sort_bm + (size_t)warp * words;
+    const int n_seg = n_tbl[0];
+    const int nw = (int)(gridDim.x * (blockDim.x >> 5));
+    for (int j = (int)blockIdx.x * (int)(blockDim.x >> 5) + warp; j < n_seg; j += nw) {
+        const int4 e = tbl[j];
+        const int m = e.z - e.y;
+        if (m >= 2) sort_segment(perm + e.y, perm + e.y, m, bm, words, lane);
     }
 }
 
@@ -238,19 +265,29 @@ __global__ void __launch_bounds__(kSumThreads, 2)
 embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, float *G, long long ld_g, const int4 *tbl,
                  const int32_t *n_tbl, const int32_t *perm)
 {
-    __shared__ float part[kSumWarps][kChunkCols];
-    griddep_wait();                             // the index kernel's table and positions
+    __shared__ float part[2][kSumWarps][kChunkCols];     // two items' partial sums, alternately
+    griddep_wait();                             // the table and the sorted positions
     const int nchunks = (H + kChunkCols - 1) / kChunkCols;
     const int total = n_tbl[0] * nchunks;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-    int4 e_next = (int)blockIdx.x < total ? tbl[blockIdx.x / nchunks] : make_int4(0, 0, 0, 0);
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+    // The next item's table entry is loaded while the current item runs, and its first batch of
+    // positions once the current item's loads are issued, so an item starts with its dY loads.
+    int4 e_next = make_int4(0, 0, 0, 0);
+    int mine_next = 0;
+    if ((int)blockIdx.x < total) {
+        e_next = tbl[blockIdx.x / nchunks];
+        const int idx = warp + kSumWarps * lane;
+        mine_next = idx < e_next.z - e_next.y ? __ldg(perm + e_next.y + idx) : 0;
+    }
+    int buf = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x, buf ^= 1) {
         const int j = item / nchunks;
         const int chunk = item - j * nchunks;
         const int4 e = e_next;                  // slot, first, end
+        const int mine_first = mine_next;
         const int nxt = item + (int)gridDim.x;
-        if (nxt < total) e_next = tbl[nxt / nchunks];   // the next item's entry, loaded early
+        if (nxt < total) e_next = tbl[nxt / nchunks];
         const int slot = e.x, b0 = e.y, n = e.z - e.y;
         const int c0 = chunk * kChunkCols + lane * 8;
         const bool col_ok = c0 < H;
@@ -260,7 +297,7 @@ embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, float *G, long long
         // loaded 8, 4, 2, 1 at a time (the count is the same for the whole warp)
         for (int base = warp; base < n; base += kSumWarps * 32) {
             const int idx = base + kSumWarps * lane;
-            const int mine = idx < n ? __ldg(perm + b0 + idx) : 0;
+            const int mine = base == warp ? mine_first : (idx < n ? __ldg(perm + b0 + idx) : 0);
             const int cnt = min(32, (n - base + kSumWarps - 1) / kSumWarps);
             int j0 = 0;
             for (; j0 + 8 <= cnt; j0 += 8) sum_batch<8>(acc, dY, ld_dy, c0, col_ok, mine, j0);
@@ -268,22 +305,26 @@ embed_sum_kernel(const uint16_t *dY, int H, long long ld_dy, float *G, long long
             if (cnt - j0 >= 2) { sum_batch<2>(acc, dY, ld_dy, c0, col_ok, mine, j0); j0 += 2; }
             if (cnt - j0 >= 1) sum_batch<1>(acc, dY, ld_dy, c0, col_ok, mine, j0);
         }
-        // fixed-order combination of the 8 warps' partial sums
+        if (nxt < total) {
+            const int idx = warp + kSumWarps * lane;
+            mine_next = idx < e_next.z - e_next.y ? __ldg(perm + e_next.y + idx) : 0;
+        }
+        // fixed-order combination of the 8 warps' partial sums; the buffers alternate, so the
+        // next item may write its partial sums while this item's are still being read
 #pragma unroll
-        for (int q = 0; q < 8; ++q) part[warp][lane * 8 + q] = acc[q];
+        for (int q = 0; q < 8; ++q) part[buf][warp][lane * 8 + q] = acc[q];
         __syncthreads();
         const int col = chunk * kChunkCols + tid;
         if (col < H) {
-            float sum = part[0][tid];
+            float sum = part[buf][0][tid];
 #pragma unroll
-            for (int w = 1; w < kSumWarps; ++w) sum = __fadd_rn(sum, part[w][tid]);
+            for (int w = 1; w < kSumWarps; ++w) sum = __fadd_rn(sum, part[buf][w][tid]);
             G[(size_t)slot * ld_g + col] = sum;
         }
-        __syncthreads();
     }
 }
 
-// The two launches of one embedding-row gradient, on scratch of scratch_ints(n_tok, slot_cap)
+// The three launches of one embedding-row gradient, on scratch of scratch_ints(n_tok, slot_cap)
 // words (16-byte aligned).
 int launch_embed(const int32_t *tokens, int n_tok, const void *dY, int H, int64_t ld_dy, const sf_mask &mk,
                  float *G, int64_t ld_g, int32_t *scratch, uint32_t *dev_status, cudaStream_t st)
@@ -294,7 +335,9 @@ int launch_embed(const int32_t *tokens, int n_tok, const void *dY, int H, int64_
     const int keep_slots = index_smem_ints(n_tok, mk.slot_cap, true) * sizeof(int) <= kSmemLimit;
     const size_t smem = index_smem_ints(n_tok, mk.slot_cap, keep_slots) * sizeof(int);
     if (smem > kSmemLimit) return SF_ERR_UNSUPPORTED;
-    if (smem > 48 * 1024 &&
+    // above 48 KB of shared memory in all, static included, the launch needs the opt-in
+    // attribute; it is set from 40 KB of dynamic memory on (the static part is far below 8 KB)
+    if (smem > 40 * 1024 &&
         cudaFuncSetAttribute(embed_index_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return SF_ERR_CUDA;
@@ -302,17 +345,24 @@ int launch_embed(const int32_t *tokens, int n_tok, const void *dY, int H, int64_
     if (sms <= 0) return SF_ERR_NO_DEVICE;
     embed_index_kernel<<<1, kIndexThreads, smem, st>>>(tokens, n_tok, mk, tbl, n_tbl, perm, keep_slots, dev_status);
     if (launch_status() != SF_OK) return SF_ERR_CUDA;
-    // the sum kernel is launched as a programmatic dependent of the index kernel: its CTAs are
-    // placed while the index kernel runs and wait for its completion before reading the table
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(sms * 4);
-    cfg.blockDim = dim3(kSumThreads);
-    cfg.stream = st;
+    // the sort and sum kernels are programmatic dependents of the kernel before them: their CTAs
+    // are placed while it runs and wait for its completion before reading what it wrote
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cfg.gridDim = dim3(sms);
+    cfg.blockDim = dim3(kSortThreads);
+    cfg.dynamicSmemBytes = (size_t)(kSortThreads / 32) * (((size_t)n_tok + 31) / 32) * sizeof(uint32_t);
+    if (cudaLaunchKernelEx(&cfg, embed_sort_kernel, static_cast<const int4 *>(tbl),
+                           static_cast<const int32_t *>(n_tbl), perm, n_tok) != cudaSuccess)
+        return SF_ERR_CUDA;
+    cfg.gridDim = dim3(sms * 4);
+    cfg.blockDim = dim3(kSumThreads);
+    cfg.dynamicSmemBytes = 0;
     if (cudaLaunchKernelEx(&cfg, embed_sum_kernel, static_cast<const uint16_t *>(dY), H, (long long)ld_dy, G,
                            (long long)ld_g, static_cast<const int4 *>(tbl), static_cast<const int32_t *>(n_tbl),
                            static_cast<const int32_t *>(perm)) != cudaSuccess)

@@ -421,7 +421,8 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
     if (n_masks == 0) return SF_OK;
     cudaStream_t st = as_stream(stream);
     const size_t fin_smem = (size_t)3 * (max_rows / 32) * sizeof(uint32_t);
-    if (fin_smem > 48 * 1024 &&
+    // opt-in beyond 48 KB of shared memory in all, static included (set from 40 KB dynamic on)
+    if (fin_smem > 40 * 1024 &&
         cudaFuncSetAttribute(mask_finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)fin_smem) != cudaSuccess)
         return SF_ERR_CUDA;

@@ -460,7 +460,8 @@ extern "C" int sf_sparse_update(const sf_matrix *mats, int n_mats, const sf_adam
 #endif
     const int unroll = SF_UPDATE_UNROLL;
     const void *fn = unroll == 2 ? (const void *)update_kernel<2> : (const void *)update_kernel<1>;
-    if (smem > 48 * 1024 &&
+    // opt-in beyond 48 KB of shared memory in all, static included (set from 40 KB dynamic on)
+    if (smem > 40 * 1024 &&
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return SF_ERR_CUDA;
     int per_sm = 0;

@@ -280,7 +280,7 @@ class StepPlan:
         else:
             n = 2 * chunks(self.n_masks, sf.SF_MASKS_PER_LAUNCH)   # accumulate + finalize per batch
         n += self.gather_launches + self.dw_launches  # row gather, then the main dW launches
-        n += 2 if self.has_emb else 0                 # embedding index, sum
+        n += 3 if self.has_emb else 0                 # embedding index, sort, sum
         n += chunks(len(self.upd_arr), sf.SF_MATS_PER_LAUNCH)
         return n
 

@@ -29,8 +29,10 @@ def _canary(shape):
 # section 2.1: masks
 # =============================================================================================
 
-def test_conductor_matches_oracle_window_by_window(sf):
-    V, cap = 1024, 256
+@pytest.mark.parametrize("V,cap", [(1024, 256), (131072, 256)])
+def test_conductor_matches_oracle_window_by_window(sf, V, cap):
+    # 131,072 rows: the finalize's shared-memory copy of the mask (3 words per 32 rows, 48 KB)
+    # needs the opt-in beyond 48 KB
     mk = sf.Mask(V, cap, DEV)
     sf.sf_mask_init(mk)
     status = sf.status_word()
@@ -376,6 +378,45 @@ def test_embed_grad_matches_oracle(sf, V, H, n):
     assert host(G2).tobytes() == got.tobytes()
 
 
+def test_embed_grad_same_bytes_in_every_index_layout(sf):
+    """The index pass keeps its working set (slots, counts, scattered positions) in shared memory
+    when it fits and otherwise moves the positions, then also the slots, to the scratch buffer;
+    at 16,384 tokens slot capacities of 4,096, 32,000 and 49,152 take the three layouts. Each
+    row's positions are sorted before the sum, so its gradient has the same bytes in all three
+    (slot numbers may differ), and matches the oracle."""
+    V, H, n = 49152, 64, 16384
+    tok = synth.zipf_ids(synth.rng(3, "tokens", V), n, V)
+    dY = synth.normal_bf16(synth.rng(3, "dy", V), (n, H))
+    priors = [synth.zipf_ids(synth.rng(3, "tokens", V, w), n, V) for w in range(3)]
+    charge = np.zeros(V, np.float32)
+    for prior in priors:
+        orc.window_tokens(charge, prior)
+    words, _ = orc.window_tokens(charge, tok)
+    ref = orc.embed_grad(tok, dY, V, words)
+    by_cap = {}
+    for cap in (4096, 32000, 49152):
+        mk = sf.Mask(V, cap, DEV)
+        sf.sf_mask_init(mk)
+        for prior in priors + [tok]:
+            sf.sf_mask_update([mk], [sf.make_src(sf.SF_SRC_TOKENS, i32_dev(prior), n=n)], 0.01)
+        mh = mask_host(mk)
+        assert np.array_equal(mh["words"], words)
+        G = _canary((cap, H))
+        ws = torch.zeros(sf.sf_embed_grad_ws_bytes(n, cap) // 4, dtype=torch.int32, device=DEV)
+        status = sf.status_word()
+        sf.sf_embed_grad(i32_dev(tok), bf16_dev(dY), mk, G, ws, status)
+        got = host(G)
+        assert host(status)[0] == 0
+        rows = mh["rows"]
+        assert 0 < len(rows) <= 4096
+        by_cap[cap] = {int(r): got[mh["row_slot"][r]].tobytes() for r in rows}
+        scale = max(np.abs(ref[rows]).max(), 1.0)
+        for r in rows:
+            e = np.abs(got[mh["row_slot"][r]].astype(np.float64) - ref[r]) / np.maximum(np.abs(ref[r]), 1e-3 * scale)
+            assert e.max() <= DW_TOL, (cap, r)
+    assert by_cap[4096] == by_cap[32000] == by_cap[49152]
+
+
 # =============================================================================================
 # sections 2.3 / 2.4: the fused sparse update
 # =============================================================================================
@@ -517,10 +558,13 @@ def test_update_coupled_pairs_and_changing_masks(sf):
     assert host(status)[0] == 0
 
 
-def test_update_wide_rows_and_overflowed_rows_untouched(sf):
-    # C = 11008 (the 7B feed-forward width) exercises several chunks per thread; slot capacity
-    # smaller than the active set: rows without a slot must not change.
-    R, C = 64, 11008
+@pytest.mark.parametrize("C", [11008, 12000])
+def test_update_wide_rows_and_overflowed_rows_untouched(sf, C):
+    # C = 11008 (the 7B feed-forward width) exercises several chunks per thread; C = 12,000 puts
+    # the row's shared-memory copy (48,000 B) plus the kernel's static shared memory just over
+    # the 48 KB that needs no opt-in. Slot capacity smaller than the active set: rows without a
+    # slot must not change.
+    R = 64
     W = synth.weights_f32(synth.rng(5, "weights"), R, C)
     words = synth.words_from_rows(R, [0, 5, 9, 33, 63])
     st = orc.MatrixState(W)
