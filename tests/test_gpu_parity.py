@@ -379,11 +379,11 @@ def test_embed_grad_matches_oracle(sf, V, H, n):
 
 
 def test_embed_grad_same_bytes_in_every_index_layout(sf):
-    """The index pass keeps its working set (slots, counts, scattered positions) in shared memory
-    when it fits and otherwise moves the positions, then also the slots, to the scratch buffer;
-    at 16,384 tokens slot capacities of 4,096, 32,000 and 49,152 take the three layouts. Each
-    row's positions are sorted before the sum, so its gradient has the same bytes in all three
-    (slot numbers may differ), and matches the oracle."""
+    """The index pass keeps each token's slot in shared memory beside the counts when both fit
+    and looks the slots up again otherwise; at 16,384 tokens, slot capacities of 4,096 and 32,000
+    keep them and 49,152 does not. Each row's positions are sorted before the sum, so its
+    gradient has the same bytes at every capacity (slot numbers may differ), and matches the
+    oracle."""
     V, H, n = 49152, 64, 16384
     tok = synth.zipf_ids(synth.rng(3, "tokens", V), n, V)
     dY = synth.normal_bf16(synth.rng(3, "dy", V), (n, H))
