@@ -1089,9 +1089,11 @@ def main():
     if "masks:accum" in pass_ms:
         hbm_kernel("mask_accum_kernel", pass_ms["masks:accum"], trk_bytes, n_mask_batches,
                    "tracker pass: Y read once, T*R*2 B per projection")
-        kern["mask_finalize_kernel"] = {"ms_per_step": pass_ms["masks:finalize"] / K,
-                                        "launches_per_step": n_mask_batches, "bound": "latency",
-                                        "note": "one CTA per mask: charges, words, lists, slots"}
+        kern["mask finalize (hmax + charge + lists)"] = {
+            "ms_per_step": pass_ms["masks:finalize"] / K, "launches_per_step": 3 * n_mask_batches,
+            "bound": "latency",
+            "note": "mask_hmax_kernel and mask_charge_kernel over 2,048-row blocks (busiest row; charges, "
+                    "words, slot changes), then mask_finalize_kernel, one CTA per mask (slots, lists)"}
         gather_bytes = sum(w["gather_bytes"] for w in work)
         main_bytes = sum(w["dw_main_bytes"] for w in work)
         hbm_kernel("dw_gather_kernel", pass_ms["masked_dw:gather"], gather_bytes, plan0.gather_launches,

@@ -71,7 +71,8 @@ typedef void *sf_stream;               /* cudaStream_t */
  *   slot_step[slot_cap]  int32  Adam step count of each slot; 0 marks fresh (zero) moments
  *   counts[8]        int32   [0] active rows, [1] active tiles, [2] free slots, [3] active rows
  *                            with no slot, [4] rows that took a fresh slot in the last call,
- *                            [5..7] reserved (zero)
+ *                            [5] used inside sf_mask_update (zero between calls), [6..7]
+ *                            reserved (zero)
  * Moments exist only for active rows (section 2.3): a row that turns active takes a free slot
  * with fresh moments, a row that turns inactive returns its slot and its moments are dropped.
  * Slot numbers are an implementation detail; compare state by row.
@@ -116,7 +117,13 @@ int sf_mask_init(const sf_mask *mk /* host */, sf_stream stream);
  * row_slot -1). `masks` and `srcs` are host arrays of n_masks entries; each entry is
  * independent. Errors: SF_ERR_ARG (shape / kind / null), SF_ERR_ALIGN, SF_ERR_UNSUPPORTED for
  * R > 262144 or slot_cap > R.
+ * Launches, per batch of up to 240 masks: the accumulate pass (TOKENS and OUTPUT sources), then
+ * the finalize: one launch (a CTA per mask), or three when a mask of the batch has
+ * SF_MASK_SPLIT_ROWS rows or more (busiest row and charge rule over 2,048-row blocks of all the
+ * batch's masks, then a CTA per mask for slots and lists), chained by programmatic dependent
+ * launch. While the finalize runs, a mask's active_tiles and tile_rows hold intermediate bits.
  */
+#define SF_MASK_SPLIT_ROWS 16384
 #define SF_SRC_TOKENS       0
 #define SF_SRC_OUTPUT_BF16  1
 #define SF_SRC_HITS_U32     2

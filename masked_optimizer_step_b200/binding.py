@@ -34,6 +34,7 @@ SF_PHASE_SECOND = 2
 
 SF_DW_MAX_PER_LAUNCH = 96
 SF_MASKS_PER_LAUNCH = 240
+SF_MASK_SPLIT_ROWS = 16384
 SF_MATS_PER_LAUNCH = 256
 
 _P = ctypes.c_void_p

@@ -8,13 +8,19 @@
 // One mask per step serves all later stages. Section 2.3 keeps optimizer moments for active
 // rows only; the slot lifecycle below is that rule.
 //
-// Two launches per call, each covering every mask of the call:
+// Four launches per call, each covering every mask of the call; the last three are chained by
+// programmatic dependent launch:
 //   mask_accum_kernel     the window's activity into accum[] -- token histogram (integer
 //                         atomics), or the column absmax of Y (16-byte loads, packed u16 max,
 //                         one atomicMax per column and CTA). HBM-bound streaming pass.
-//   mask_finalize_kernel  one CTA per mask: busiest row, charge update, ballot into mask words,
-//                         slot release / allocation in ascending row order, ordered lists.
-// Both reductions are order-free (integer adds, max), so masks and lists are bit-exact.
+//   mask_hmax_kernel      the busiest row of each mask: 2,048-row blocks, one atomicMax each.
+//   mask_charge_kernel    the charge update and the new mask words, 2,048-row blocks, and per
+//                         32-row tile the rows that release a slot or need one.
+//   mask_finalize_kernel  one CTA per mask: slot release / allocation in ascending row order,
+//                         ordered lists.
+// The reductions are order-free (integer adds, max), so masks and lists are bit-exact. A large
+// mask's per-row work is spread over many SMs by the middle two launches: one CTA reading and
+// writing a 32,000-row mask's state is bound by one SM's memory throughput (~20 us).
 #include "sf_common.cuh"
 #include "sf_host.h"
 
@@ -49,6 +55,7 @@ struct MaskDesc {
     int32_t *slot_step;
     int32_t *counts;
     int32_t cta_begin;    // first CTA of this mask in the accumulate launch
+    int32_t blk_begin;    // first 2,048-row block of this mask in the hmax and charge launches
     int32_t col_blocks;   // OUTPUT: 2048-column blocks
     int32_t tok_segs;     // OUTPUT: token segments
 };
@@ -58,6 +65,7 @@ constexpr int kMaxMasksPerLaunch = 240;
 struct MaskBatch {
     int32_t n;
     int32_t total_ctas;
+    int32_t total_blks;
     MaskDesc d[kMaxMasksPerLaunch];
 };
 static_assert(sizeof(MaskBatch) <= 32764, "kernel parameter space");
@@ -68,6 +76,16 @@ __device__ __forceinline__ int find_mask(const MaskBatch &b, int cta)
     while (lo < hi) {
         int mid = (lo + hi + 1) >> 1;
         if (b.d[mid].cta_begin <= cta) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ int find_mask_blk(const MaskBatch &b, int blk)
+{
+    int lo = 0, hi = b.n - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (b.d[mid].blk_begin <= blk) lo = mid; else hi = mid - 1;
     }
     return lo;
 }
@@ -171,49 +189,62 @@ mask_accum_kernel(const __grid_constant__ MaskBatch b, uint32_t *status)
     }
 }
 
-// Finalize, one CTA per mask. Phase 2 runs one warp per 32-row tile (lane = row) and issues the
-// loads of kBatch tiles before using any of them, so a warp has several independent DRAM round
-// trips in flight (32 registers: two CTAs per SM, so 296 masks finalize in one wave); the new, released and needing-a-slot bit masks of every tile stay in shared
-// memory. The slot sweeps and the lists then go over rounds of kRound words: a block scan of the
-// per-word counts gives every tile its offsets, and a warp per tile writes its rows' entries,
-// touching global memory only for rows that change state.
+// The busiest row, the charge rule and the new words run over 2,048-row blocks (256 threads: a
+// warp per 32-row tile, lane = row, the loads of kBatch tiles issued before any is used); the
+// finalize then runs one CTA per mask over the bit masks they leave: new words in words[],
+// the rows that release a slot in active_tiles[] and those that need one in tile_rows[] (one
+// uint32 per tile; both arrays are rewritten with the lists afterwards). The slot sweeps and the
+// lists go over rounds of kRound words: a block scan of the per-word counts gives every tile its
+// offsets, and a warp per tile writes its rows' entries, touching global memory only for rows
+// that change state. The busiest row's value meets in counts[5] (reset by the finalize).
+constexpr int kBlkThreads = 256;
+constexpr int kBlkRows = 2048;
+constexpr int kSplitRows = SF_MASK_SPLIT_ROWS;   // masks from this many rows on take the split finalize
+constexpr int kBlkWords = kBlkRows / 32;
 constexpr int kBatch = 4;
 constexpr int kRound = 512;       // words per scan round; per-round sums stay below 2^15 per field
 
-__global__ void __launch_bounds__(kFinalizeThreads, 2)   // two per SM: a call's masks fit one wave
-mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *status)
+__global__ void __launch_bounds__(kBlkThreads)
+mask_hmax_kernel(const __grid_constant__ MaskBatch b)
 {
-    extern __shared__ uint32_t smem_words[];
-    __shared__ int scan_scratch[33];
+    griddep_launch_dependents();
+    griddep_wait();                           // the window's activity
     __shared__ uint32_t max_scratch[33];
-    __shared__ int s_off[kRound];
-    __shared__ int s_toff[kRound];
-
-    const MaskDesc &d = b.d[blockIdx.x];
-    const int R = d.R, nw = R >> 5;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int nwarps = kFinalizeThreads / 32;
-    const uint32_t lt = (1u << lane) - 1u;
-    uint32_t *new_w = smem_words;
-    uint32_t *rel_w = smem_words + nw;
-    uint32_t *need_w = smem_words + 2 * nw;
-    const int kind = d.kind;
-    const uint32_t *src_u32 = static_cast<const uint32_t *>(d.src);
-
-    // (1) busiest row of the window
+    const int i = find_mask_blk(b, blockIdx.x);
+    const MaskDesc &d = b.d[i];
+    if (d.kind == SF_SRC_WORDS) return;
+    const uint32_t *vals = d.kind == SF_SRC_HITS_U32 ? static_cast<const uint32_t *>(d.src) : d.accum;
+    const int r0 = (blockIdx.x - d.blk_begin) * kBlkRows;
+    const int r1 = min(d.R, r0 + kBlkRows);
     uint32_t hmax = 0;
-    if (kind == SF_SRC_TOKENS || kind == SF_SRC_OUTPUT_BF16) {
-#pragma unroll 4
-        for (int r = tid; r < R; r += kFinalizeThreads) hmax = max(hmax, d.accum[r]);
-    } else if (kind == SF_SRC_HITS_U32) {
-#pragma unroll 4
-        for (int r = tid; r < R; r += kFinalizeThreads) hmax = max(hmax, src_u32[r]);
+    if ((reinterpret_cast<uintptr_t>(vals) & 15) == 0) {
+        // rows come in whole 32-row tiles, so each thread's four-row groups stay in the block
+#pragma unroll
+        for (int u = 0; u < kBlkRows / (4 * kBlkThreads); ++u) {
+            const int r = r0 + 4 * (u * kBlkThreads + (int)threadIdx.x);
+            if (r < r1) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(vals + r);
+                hmax = max(hmax, max(max(v.x, v.y), max(v.z, v.w)));
+            }
+        }
+    } else {                                  // a caller's hit counts need only 4-byte alignment
+        for (int r = r0 + (int)threadIdx.x; r < r1; r += kBlkThreads) hmax = max(hmax, vals[r]);
     }
     hmax = block_max_u32(hmax, max_scratch);
-    const float H = kind == SF_SRC_OUTPUT_BF16 ? __uint_as_float(hmax) : __uint2float_rn(hmax);
+    if (threadIdx.x == 0 && hmax) atomicMax(reinterpret_cast<unsigned int *>(&d.counts[5]), hmax);
+}
 
-    // (2) charge rule, new mask word, and which rows release or need a slot
-    for (int w0 = warp; w0 < nw; w0 += nwarps * kBatch) {
+// The charge rule and the new mask words of tiles [w_begin, w_end) of one mask, a warp per tile
+// (w = w_begin + warp, + nwarps, ...); per tile the new word and the rows that release a slot or
+// need one go to new_w[w], rel_w[w], need_w[w] (shared memory, or the mask's own arrays).
+__device__ __forceinline__ void charge_words(const MaskDesc &d, int w_begin, int w_end, int warp, int nwarps,
+                                             float H, float thr, uint32_t *new_w, uint32_t *rel_w,
+                                             uint32_t *need_w)
+{
+    const int lane = threadIdx.x & 31;
+    const int kind = d.kind;
+    const uint32_t *src_u32 = static_cast<const uint32_t *>(d.src);
+    for (int w0 = w_begin + warp; w0 < w_end; w0 += nwarps * kBatch) {
         uint32_t hv[kBatch], ow[kBatch];
         float qv[kBatch];
         int sl[kBatch];
@@ -224,7 +255,7 @@ mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *s
             ow[k] = 0u;
             qv[k] = 0.0f;
             sl[k] = -1;
-            if (w < nw) {
+            if (w < w_end) {
                 const int r = (w << 5) + lane;
                 if (kind == SF_SRC_WORDS) {
                     hv[k] = src_u32[w];
@@ -239,7 +270,7 @@ mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *s
 #pragma unroll
         for (int k = 0; k < kBatch; ++k) {
             const int w = w0 + k * nwarps;
-            if (w >= nw) break;                                  // uniform across the warp
+            if (w >= w_end) break;                               // uniform across the warp
             const int r = (w << 5) + lane;
             bool act;
             if (kind == SF_SRC_WORDS) {
@@ -261,6 +292,65 @@ mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *s
                 rel_w[w] = rel;
                 need_w[w] = need;
             }
+        }
+    }
+}
+
+__device__ __forceinline__ float busiest_value(const MaskDesc &d, uint32_t hmax)
+{
+    return d.kind == SF_SRC_OUTPUT_BF16 ? __uint_as_float(hmax) : __uint2float_rn(hmax);
+}
+
+__global__ void __launch_bounds__(kBlkThreads)
+mask_charge_kernel(const __grid_constant__ MaskBatch b, float thr)
+{
+    griddep_launch_dependents();
+    griddep_wait();                           // the busiest row
+    const int i = find_mask_blk(b, blockIdx.x);
+    const MaskDesc &d = b.d[i];
+    const int w_begin = (blockIdx.x - d.blk_begin) * kBlkWords;
+    const int w_end = min(d.R >> 5, w_begin + kBlkWords);
+    const float H = busiest_value(d, static_cast<uint32_t>(d.counts[5]));
+    charge_words(d, w_begin, w_end, threadIdx.x >> 5, kBlkThreads / 32, H, thr, d.words,
+                 reinterpret_cast<uint32_t *>(d.active_tiles), reinterpret_cast<uint32_t *>(d.tile_rows));
+}
+
+// fused = 1: the CTA also finds the busiest row and runs the charge rule itself (one launch; the
+// masks of the call are small enough for one SM each); fused = 0: mask_hmax_kernel and
+// mask_charge_kernel ran first and left the bit masks in the mask's arrays.
+__global__ void __launch_bounds__(kFinalizeThreads, 2)   // two per SM: a call's masks fit one wave
+mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, int fused, uint32_t *status)
+{
+    griddep_launch_dependents();
+    extern __shared__ uint32_t smem_words[];
+    __shared__ int scan_scratch[33];
+    __shared__ uint32_t max_scratch[33];
+    __shared__ int s_off[kRound];
+    __shared__ int s_toff[kRound];
+
+    const MaskDesc &d = b.d[blockIdx.x];
+    const int R = d.R, nw = R >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int nwarps = kFinalizeThreads / 32;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t *new_w = smem_words;
+    uint32_t *rel_w = smem_words + nw;
+    uint32_t *need_w = smem_words + 2 * nw;
+    griddep_wait();                           // the window's activity, or the charge pass's bit masks
+    if (fused) {
+        uint32_t hmax = 0;
+        if (d.kind != SF_SRC_WORDS) {
+            const uint32_t *vals = d.kind == SF_SRC_HITS_U32 ? static_cast<const uint32_t *>(d.src) : d.accum;
+#pragma unroll 4
+            for (int r = tid; r < R; r += kFinalizeThreads) hmax = max(hmax, vals[r]);
+        }
+        hmax = block_max_u32(hmax, max_scratch);
+        charge_words(d, 0, nw, warp, nwarps, busiest_value(d, hmax), thr, new_w, rel_w, need_w);
+    } else {
+        for (int w = tid; w < nw; w += kFinalizeThreads) {
+            new_w[w] = d.words[w];
+            rel_w[w] = static_cast<uint32_t>(d.active_tiles[w]);
+            need_w[w] = static_cast<uint32_t>(d.tile_rows[w]);
         }
     }
     __syncthreads();
@@ -342,6 +432,7 @@ mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, uint32_t *s
         d.counts[2] = max(top2 - need_base, 0);
         d.counts[3] = total_over;
         d.counts[4] = min(need_base, top2);
+        d.counts[5] = 0;                      // the busiest row's meeting point, for the next window
         if (total_over) set_status(status, SF_STATUS_SLOT_OVERFLOW);
     }
 }
@@ -448,7 +539,7 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
         }
         MaskBatch batch;
         batch.n = cnt;
-        int ctas = 0;
+        int ctas = 0, blks = 0;
         for (int j = 0; j < cnt; ++j) {
             const sf_mask &m = masks[first + j];
             const sf_mask_src &s = srcs[first + j];
@@ -470,6 +561,8 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
             d.slot_step = m.slot_step;
             d.counts = m.counts;
             d.cta_begin = ctas;
+            d.blk_begin = blks;
+            blks += (m.R + kBlkRows - 1) / kBlkRows;
             d.col_blocks = (m.R + kColsPerCta - 1) / kColsPerCta;
             d.tok_segs = (s.n + seg_tokens - 1) / seg_tokens;
             if (s.kind == SF_SRC_TOKENS)
@@ -478,13 +571,36 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
                 ctas += d.col_blocks * d.tok_segs;
         }
         batch.total_ctas = ctas;
+        batch.total_blks = blks;
         if (ctas > 0 && phase != SF_PHASE_SECOND) {
             mask_accum_kernel<<<ctas, kAccumThreads, 0, st>>>(batch, dev_status);
             if (launch_status() != SF_OK) return SF_ERR_CUDA;
         }
         if (phase != SF_PHASE_FIRST) {
-            mask_finalize_kernel<<<cnt, kFinalizeThreads, fin_smem, st>>>(batch, threshold, dev_status);
-            if (launch_status() != SF_OK) return SF_ERR_CUDA;
+            // one launch when every mask of the batch is small enough for one SM; otherwise the
+            // busiest row and the charge rule go over 2,048-row blocks first
+            int batch_max_rows = 0;
+            for (int j = 0; j < cnt; ++j) batch_max_rows = max(batch_max_rows, masks[first + j].R);
+            const int fused = batch_max_rows < kSplitRows;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[0].val.programmaticStreamSerializationAllowed = 1;
+            cudaLaunchConfig_t cfg = {};
+            cfg.stream = st;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (!fused) {
+                cfg.gridDim = dim3(blks);
+                cfg.blockDim = dim3(kBlkThreads);
+                if (cudaLaunchKernelEx(&cfg, mask_hmax_kernel, batch) != cudaSuccess) return SF_ERR_CUDA;
+                if (cudaLaunchKernelEx(&cfg, mask_charge_kernel, batch, threshold) != cudaSuccess)
+                    return SF_ERR_CUDA;
+            }
+            cfg.gridDim = dim3(cnt);
+            cfg.blockDim = dim3(kFinalizeThreads);
+            cfg.dynamicSmemBytes = fin_smem;
+            if (cudaLaunchKernelEx(&cfg, mask_finalize_kernel, batch, threshold, fused, dev_status) != cudaSuccess)
+                return SF_ERR_CUDA;
         }
     }
     return SF_OK;

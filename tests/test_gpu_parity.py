@@ -133,9 +133,15 @@ def test_tracker_non_finite_outputs_match_oracle(sf):
         assert (n_bad > 0) == (plant != "finite")
 
 
-def test_many_masks_in_one_call_and_explicit_sources(sf):
+@pytest.mark.parametrize("specs", [
+    [(1024, "tokens"), (4096, "output"), (256, "words"), (512, "hits"), (11008, "output")],
+    # a mask of 16,384 rows or more sends the whole batch through the three-launch finalize;
+    # the hit counts start 4 bytes past a 16-byte boundary
+    [(1024, "tokens"), (4096, "output"), (256, "words"), (32768, "hits+4"), (11008, "output"),
+     (16384, "tokens")],
+])
+def test_many_masks_in_one_call_and_explicit_sources(sf, specs):
     # several masks of different kinds and sizes in one call, each independent
-    specs = [(1024, "tokens"), (4096, "output"), (256, "words"), (512, "hits"), (11008, "output")]
     masks, srcs, keep, ref = [], [], [], []
     for i, (R, kind) in enumerate(specs):
         mk = sf.Mask(R, R // 2, DEV)
@@ -159,7 +165,11 @@ def test_many_masks_in_one_call_and_explicit_sources(sf):
         else:
             tok = synth.zipf_ids(g, 300, R)
             hits = np.bincount(tok, minlength=R).astype(np.uint32)
-            t = u32_dev(hits)
+            if kind == "hits+4":
+                t = u32_dev(np.concatenate([np.zeros(1, np.uint32), hits]))[1:]
+                assert t.data_ptr() % 16 == 4
+            else:
+                t = u32_dev(hits)
             srcs.append(sf.make_src(sf.SF_SRC_HITS_U32, t))
             words, _ = orc.window_tokens(charge, tok)      # same counts, folded by the oracle
         keep.append(t)
