@@ -55,6 +55,39 @@ def test_embed_grad_with_no_active_row_writes_nothing(sf):
     assert (host(G).view(np.uint32) == CANARY).all()
 
 
+@pytest.mark.parametrize("case", ["one row takes every token", "every token its own row"])
+def test_embed_grad_segment_extremes(sf, case):
+    """The segment sort at its extremes: a single segment of the largest length (16,384
+    positions, a 512-word bitmap, in place) and 2,048 segments of one position each."""
+    H = 64
+    if case == "one row takes every token":
+        V, n, rows = 1024, 16384, [517]
+        tok = np.full(n, 517, np.int32)
+        tok[::7] = 3                              # an inactive row in between
+    else:
+        V, n = 4096, 2048
+        tok = synth.rng(6, "tokens").permutation(V)[:n].astype(np.int32)
+        rows = np.sort(tok)
+    cap = max(32, len(rows))
+    mk = _words_mask(sf, V, cap, rows)
+    dY = synth.normal_bf16(synth.rng(6, "dy", n), (n, H))
+    G = _canary((cap, H))
+    ws = torch.zeros(sf.sf_embed_grad_ws_bytes(n, cap) // 4, dtype=torch.int32, device=DEV)
+    status = sf.status_word()
+    sf.sf_embed_grad(i32_dev(tok), bf16_dev(dY), mk, G, ws, status)
+    mh = mask_host(mk)
+    ref = orc.embed_grad(tok, dY, V, mh["words"])
+    got = host(G)
+    scale = max(np.abs(ref[mh["rows"]]).max(), 1.0)
+    for r in mh["rows"]:
+        e = np.max(np.abs(got[mh["row_slot"][r]] - ref[r]) / np.maximum(np.abs(ref[r]), 1e-3 * scale))
+        assert e <= 2e-3, int(r)
+    assert int(host(status)[0]) == 0
+    G2 = _canary((cap, H))                        # the same bytes again
+    sf.sf_embed_grad(i32_dev(tok), bf16_dev(dY), mk, G2, ws)
+    assert host(G2).tobytes() == got.tobytes()
+
+
 def _matrix(sf, R, C, cap, seed):
     W = synth.weights_f32(synth.rng(seed, "weights"), R, C)
     mat = sf.Matrix(R, C, cap, DEV)
