@@ -522,8 +522,11 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
     for (int first = 0; first < n_masks; first += kMaxMasksPerLaunch) {
         const int cnt = n_masks - first < kMaxMasksPerLaunch ? n_masks - first : kMaxMasksPerLaunch;
         // Token segment length of the column-absmax pass: 512 tokens, shortened (down to 32) when
-        // the launch would otherwise give each SM fewer than ~8 CTAs, so that enough loads are in
-        // flight to cover HBM latency (a lone projection has only R / 2048 column blocks).
+        // the launch would otherwise give each SM fewer than ~2 CTAs, so that enough loads are in
+        // flight to cover HBM latency (a lone projection has only R / 2048 column blocks). Each
+        // segment ends in one atomicMax per column, so shorter segments cost atomics: for one 7B
+        // layer at 4,096 tokens the pass measured fastest at ~2 CTAs per SM (4: +2 us, 8: +7 us,
+        // 16: +35 us).
         int seg_tokens = kTokensPerSeg;
         {
             long base = 0;
@@ -533,7 +536,7 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
                     base += (long)((masks[first + j].R + kColsPerCta - 1) / kColsPerCta) *
                             ((s.n + kTokensPerSeg - 1) / kTokensPerSeg);
             }
-            const long target = 8L * (sms > 0 ? sms : 148);
+            const long target = 2L * (sms > 0 ? sms : 148);
             while (base > 0 && seg_tokens > kMinTokensPerSeg && base * (kTokensPerSeg / seg_tokens) < target)
                 seg_tokens >>= 1;
         }
