@@ -6,8 +6,10 @@
 // bit is clear inside a live tile are dropped when the result is written out.
 //
 // Shapes: dX is T x R (token-major; column r is weight row r), A is T x C (token-major). In
-// GEMM terms M = weight rows, N = columns, K = tokens, and BOTH operands are M/N-contiguous
-// ("MN-major"): tcgen05 reads them that way directly, so nothing is transposed in memory.
+// GEMM terms M = weight rows, N = columns, K = tokens. A (the B operand) is read in place,
+// N-contiguous ("MN-major"); tile mode reads dX's tiles in place too (M-contiguous), while row
+// mode's gather stores each gathered row's tokens contiguously (K-major). tcgen05 reads both
+// layouts directly, so nothing else is transposed.
 //
 // Groups. Consecutive problems of a call that read the same A (same pointer, stride, C and T --
 // e.g. the q, k and v projections of a layer, or gate and up) form a group: their rows share
@@ -17,14 +19,16 @@
 //              cut into 128-row M-tiles of four tiles, gathered straight from dX by TMA; rows of
 //              a live tile that are inactive are computed and dropped at the store.
 //   row mode   a gather kernel first copies just the active rows of every problem of the group
-//              into a dense token-major buffer (caller scratch), so an M-tile holds 128 active
-//              rows instead of four tiles. Same result; far fewer tensor-core FLOPs when rows are
+//              into a dense buffer (caller scratch; each row's tokens contiguous), so an M-tile
+//              holds 128 active rows instead of four tiles. Same result; far fewer tensor-core FLOPs when rows are
 //              scattered (at 1% scattered rows, a live tile holds ~1.2 active rows).
 // Row mode is used when the group's active rows fit the scratch and it needs fewer M-tiles.
 //
 // CTA (1 per SM, 320 threads, warp-specialised, persistent over the units of the launch):
-//   warp 0      TMA producer: per 64-token stage, four 32-row boxes of the A-operand
-//               (SWIZZLE_64B) and four 64-column boxes of A (SWIZZLE_128B) into a 4-deep ring;
+//   warp 0      TMA producer: per 64-token stage, the A-operand -- four 32-row boxes of dX
+//               (tile mode, SWIZZLE_64B) or one {64 tokens, 128 rows} box of the gathered rows
+//               (row mode, SWIZZLE_128B) -- and the stage's four 64-column chunks of A in one
+//               3-D box (SWIZZLE_128B), into a 4-deep ring;
 //   warp 1      allocates 512 TMEM columns, one thread issues tcgen05.mma kind::f16
 //               (M=128, N=256, K=16, bf16 in, fp32 accumulate). Each chunk of 1024 tokens goes
 //               into one of two 256-column TMEM buffers, starting from zero; the thread commits
