@@ -145,6 +145,17 @@ def dw_gather_launch_count(problems, max_groups=192, max_probs=384, max_per_grou
     return launches
 
 
+def mask_launch_count(rows) -> int:
+    """Launches of one sf_mask_update call over masks of the given row counts (all sources that
+    accumulate: tokens or outputs). Per batch of SF_MASKS_PER_LAUNCH masks: the accumulate pass,
+    then a one-launch finalize, or a three-launch one (busiest row, charges, lists) when the batch
+    holds a mask of SF_MASK_SPLIT_ROWS rows or more."""
+    k, n = sf.SF_MASKS_PER_LAUNCH, 0
+    for b in range(0, len(rows), k):
+        n += 1 + (3 if max(rows[b:b + k]) >= sf.SF_MASK_SPLIT_ROWS else 1)
+    return n
+
+
 class StepPlan:
     """ABI argument arrays of one step over `model` for one set of input buffers.
 
@@ -276,21 +287,12 @@ class StepPlan:
         def chunks(n, k):
             return (n + k - 1) // k
 
-        def mask_call(rows):
-            # per batch of masks: the accumulate pass, then a one-launch finalize, or a three-launch
-            # one (busiest row, charges, lists) when the batch holds a mask of SF_MASK_SPLIT_ROWS
-            # rows or more
-            k, n = sf.SF_MASKS_PER_LAUNCH, 0
-            for b in range(0, len(rows), k):
-                n += 1 + (3 if max(rows[b:b + k]) >= sf.SF_MASK_SPLIT_ROWS else 1)
-            return n
-
         rows = [m.mask.R for m in ([self.model.emb] if self.has_emb else [])] + \
             [p.mat.mask.R for p in self.model.projs[self.i0:self.i1]]
         if split_embedding and self.has_emb:         # conductor and trackers as two calls
-            n = mask_call(rows[:1]) + (mask_call(rows[1:]) if len(rows) > 1 else 0)
+            n = mask_launch_count(rows[:1]) + (mask_launch_count(rows[1:]) if len(rows) > 1 else 0)
         else:
-            n = mask_call(rows)
+            n = mask_launch_count(rows)
         n += self.gather_launches + self.dw_launches  # row gather, then the main dW launches
         n += 3 if self.has_emb else 0                 # embedding index, sort, sum
         n += chunks(len(self.upd_arr), sf.SF_MATS_PER_LAUNCH)
