@@ -26,9 +26,10 @@
 //
 // CTA (1 per SM, 320 threads, warp-specialised, persistent over the units of the launch):
 //   warp 0      TMA producer: per 64-token stage, the A-operand -- four 32-row boxes of dX
-//               (tile mode, SWIZZLE_64B) or one {64 tokens, 128 rows} box of the gathered rows
-//               (row mode, SWIZZLE_128B) -- and the stage's four 64-column chunks of A in one
-//               3-D box (SWIZZLE_128B), into a 4-deep ring;
+//               (tile mode, SWIZZLE_64B) or up to four {64 tokens, 32 rows} boxes of the
+//               gathered rows, only those holding rows (row mode, SWIZZLE_128B) -- and the
+//               stage's four 64-column chunks of A in one 3-D box (SWIZZLE_128B), into a 4-deep
+//               ring;
 //   warp 1      allocates 512 TMEM columns, one thread issues tcgen05.mma kind::f16
 //               (M=128, N=256, K=16, bf16 in, fp32 accumulate). Each chunk of 1024 tokens goes
 //               into one of two 256-column TMEM buffers, starting from zero; the thread commits
@@ -115,8 +116,9 @@ struct alignas(64) DwGroup {
     // layout the four 2-D boxes give); otherwise 2-D {C, T}, box {64, 64}. 128-byte swizzle.
     CUtensorMap tm_a;
     // gathered rows, stored row by row (each row's tokens contiguous, stride tp): 2-D {T, mcap},
-    // box {64 tokens, 128 rows}, 128-byte swizzle -- a K-major operand, as the tensor cores read
-    // fastest; tokens from T to tp are outside the map and read as zeros
+    // box {64 tokens, 32 rows}, 128-byte swizzle -- a K-major operand, as the tensor cores read
+    // fastest; tokens from T to tp are outside the map and read as zeros. A stage loads only the
+    // 32-row boxes that hold gathered rows of the CTA's M-tile
     CUtensorMap tm_g;
     const int32_t *info;         // device: [0] mode (1 = rows), [1] gathered rows (null: tiles only)
     const int32_t *rowmap;       // device: per gathered row, (slot << 3) | problem, or -1
@@ -414,11 +416,16 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 const CUtensorMap *tm_rows;
                 int coord[4];
                 int nvalid = 0;
-                if (x.rows_mode) {                  // one K-major box: the CTA's 128 gathered rows
+                if (x.rows_mode) {
+                    // K-major 32-row boxes of the CTA's gathered rows, as many as hold rows: the
+                    // MMA also reads the rest of the 128-row operand (whatever an earlier stage
+                    // left), which only feeds accumulator rows the epilogue discards
                     tm_rows = &g.tm_g;
-                    coord[0] = x.mt * UM + (int)crank * BM;
-                    coord[1] = coord[2] = coord[3] = -1;
-                    nvalid = 4;
+                    const int r0 = x.mt * UM + (int)crank * BM;
+                    const int n_here = min(BM, max(0, g.info[1] - r0));
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) coord[s] = 32 * s < n_here ? r0 + 32 * s : -1;
+                    nvalid = (n_here + 31) / 32;
                 } else {
                     const DwProb &p = prb(b, x.p);
                     tm_rows = &p.tm_dx;
@@ -436,7 +443,7 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                 if (PAIR == 2 && leader) {
 #pragma unroll
                     for (int s = 0; s < 4; ++s) {
-                        if (x.rows_mode) nvalid_peer += 1;
+                        if (x.rows_mode) nvalid_peer += x.mt * UM + BM + 32 * s < g.info[1];
                         else nvalid_peer += x.mt * UNIT_TILES + 4 + s < prb(b, x.p).counts[1];
                     }
                 }
@@ -451,8 +458,12 @@ masked_dw_kernel(const __grid_constant__ DwBatch b, uint32_t *status)
                     const bool withhold = b.withhold_test && blockIdx.x == 0 && u == unit0 && kb == 0;
                     if (!withhold) {
                         if (x.rows_mode) {
-                            if (PAIR == 2) tma_load_2d_pair(sa, tm_rows, &full_bar[stage], kb * BK, coord[0]);
-                            else tma_load_2d(sa, tm_rows, &full_bar[stage], kb * BK, coord[0]);
+#pragma unroll
+                            for (int s = 0; s < 4; ++s)
+                                if (coord[s] >= 0) {
+                                    if (PAIR == 2) tma_load_2d_pair(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], kb * BK, coord[s]);
+                                    else tma_load_2d(sa + s * A_TILE_BYTES, tm_rows, &full_bar[stage], kb * BK, coord[s]);
+                                }
                         } else {
 #pragma unroll
                             for (int s = 0; s < 4; ++s)
@@ -691,7 +702,7 @@ bool encode_rows_kmajor(CUtensorMap *m, const void *base, int T, int mcap, int64
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)T, (cuuint64_t)mcap};
     const cuuint64_t strides[1] = {(cuuint64_t)tp * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, 32u};
     const cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
