@@ -295,6 +295,38 @@ def test_masked_dw_deterministic(sf, mode):
     assert a.tobytes() == host(case["dW"]).tobytes()
 
 
+@pytest.mark.parametrize("T,R,C,kind", [
+    (4096, 256, 512, "scattered"),    # 2 units of 64 token stages (four accumulation chunks each)
+    (130, 1280, 256, "scattered"),    # 3 stages per unit, ragged T
+    (1000, 4096, 2048, "clustered"),  # ~80 units of 16 stages in tile mode
+    (2048, 11008, 4096, "scattered"),  # 7B gate-like shape at 1%: row mode
+])
+def test_masked_dw_workspace_calls_are_repeatable(sf, T, R, C, kind):
+    # The call with a workspace (the device picks row or tile mode) against the oracle, byte-equal
+    # over two calls whatever the scratch held before, and close to the mask-tile launch without
+    # a workspace (the same sums).
+    g = synth.rng(31, "rows", T, R)
+    rows = synth.scattered_rows(g, R, 0.01 if R > 4096 else 0.15) if kind == "scattered" \
+        else synth.clustered_rows(g, R, 0.3)
+    case = _dw_case(sf, T, R, C, rows, 31)
+    p = [sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])]
+    status = sf.status_word()
+    ws = sf.dw_workspace(p)
+    sf.sf_masked_dw(p, status, ws=ws)
+    _check_dw(case)
+    a = host(case["dW"]).copy()
+    ws.fill_(0x5A)                          # stale scratch contents do not matter
+    sf.sf_masked_dw(p, status, ws=ws)
+    assert a.tobytes() == host(case["dW"]).tobytes()
+    sf.sf_masked_dw(p, status)              # whole units (mask-tile mode)
+    mh = mask_host(case["mask"])
+    b = host(case["dW"])
+    for r in mh["rows"]:
+        s_ = mh["row_slot"][r]
+        assert rel_err(a[s_], b[s_], 1e-2) <= 1e-4, r    # the same sums in another order
+    assert host(status)[0] == 0
+
+
 def test_masked_dw_groups_share_inputs_and_pick_their_mode(sf):
     # q/k/v-like problems reading one A (a group: their scattered rows share 128-row tiles), a
     # gate/up-like pair with whole active tiles (2 M-tiles either way, so tile mode is kept), and
@@ -792,3 +824,24 @@ def test_masked_dw_wait_timeout_is_reported_and_the_context_survives(sf, monkeyp
     for r in mh["rows"]:
         s = mh["row_slot"][r]
         assert rel_err(got[s], ref[r]) <= DW_TOL, r
+
+
+def test_masked_dw_wait_timeout_with_workspace_leaves_the_next_call_correct(sf, monkeypatch):
+    # The same bounded-wait path in a call with a workspace (row mode): after the timeout the
+    # next call on the same workspace is correct.
+    R, C, T = 1280, 512, 1024
+    rows = synth.scattered_rows(synth.rng(32, "rows"), R, 0.2)
+    case = _dw_case(sf, T, R, C, rows, 32)
+    p = [sf.dw_problem(case["dXd"], case["Ad"], case["mask"], case["dW"])]
+    ws = sf.dw_workspace(p)
+    status = sf.status_word()
+    monkeypatch.setenv("SF_TEST_DW_WITHHOLD", "1")
+    sf.sf_masked_dw(p, status, ws=ws)
+    torch.cuda.synchronize()
+    assert int(host(status)[0]) & sf.SF_STATUS_WAIT_TIMEOUT
+    monkeypatch.delenv("SF_TEST_DW_WITHHOLD")
+    status2 = sf.status_word()
+    case["dW"].view(torch.int32).fill_(int(CANARY))
+    sf.sf_masked_dw(p, status2, ws=ws)
+    assert int(host(status2)[0]) == 0
+    _check_dw(case)
