@@ -65,14 +65,15 @@ static_assert(sizeof(UpdBatch) <= 32764, "kernel parameter space");
 // product is within 1.6e-5 of W / s and the rounded quotient within 7.6e-6 (|W / s| <= 127.5),
 // so the two differ by less than 2.3e-5 and can only round differently when the product lies
 // that close to a half-integer. The exact division is taken whenever the product lies within
-// 2^-14 (about 6.1e-5) of a half-integer: a band chosen wider than the 2.3e-5 bound on purpose
-// (about 1 element in 8,000 takes it).
+// 2^-14 (about 6.1e-5) of a half-integer, i.e. farther than 0.5 - 2^-14 from the nearest
+// integer: a band chosen wider than the 2.3e-5 bound on purpose (about 1 element in 8,000 takes
+// it). y - rint(y) is exact for these magnitudes.
 __device__ __forceinline__ float quant_code(float w, float sp, float rcp, bool fast)
 {
     float qf;
     const float y = __fmul_rn(w, rcp);
-    const float frac = y - floorf(y);
-    if (fast && fabsf(frac - 0.5f) >= 0x1p-14f) qf = rintf(y);
+    const float r = rintf(y);
+    if (fast && fabsf(y - r) <= 0.5f - 0x1p-14f) qf = r;
     else qf = rintf(__fdiv_rn(w, sp));
     return fminf(fmaxf(qf, -127.0f), 127.0f);
 }
@@ -111,7 +112,7 @@ struct AdamRow {
     float sc, c_self, c_partner, beta1, beta2, omb1, omb2, bc1, bc2, eps, nlr, nlrwd, clip, wd;
 };
 
-// nan_sum stays exactly 0 while every new weight is finite (w - w is 0 for finite w, NaN for
+// nan_sum stays exactly 0 while every new weight is finite (w * 0 is 0 for finite w, NaN for
 // inf or NaN, and a NaN survives every later addition); big tracks the largest moment, which
 // must stay below 65520 to be representable in fp16.
 __device__ __forceinline__ void adam_chunk(const Chunk &k, const AdamRow &a, float (&wn)[8], uint4 &mo,
@@ -149,7 +150,7 @@ __device__ __forceinline__ void adam_chunk(const Chunk &k, const AdamRow &a, flo
             if (a.wd != 0.0f) Wn = __fmaf_rn(a.nlrwd, W, Wn);
             wn[e] = Wn;
             amax = fmaxf(amax, fabsf(Wn));
-            nan_sum = __fadd_rn(nan_sum, __fsub_rn(Wn, Wn));
+            nan_sum = __fmaf_rn(Wn, 0.0f, nan_sum);
             big = fmaxf(big, fmaxf(fabsf(m1[h]), v1[h]));
         }
         const __half2 mh = __floats2half2_rn(m1[0], m1[1]);
