@@ -60,7 +60,10 @@ typedef void *sf_stream;               /* cudaStream_t */
  * Row-mask state of one matrix (an embedding table or a projection). All arrays are device
  * memory owned by the caller; sf_mask_init() puts them in their starting state.
  *   charge[R]        float   per-row charge q_r of the charge rule (section 2.1)
- *   accum[R]         uint32  per-window accumulator; the library keeps it zero between calls
+ *   accum[R]         uint32  per-window accumulator; the library keeps it zero between calls.
+ *                            Token sources count hits in it, one uint32 per row; output sources
+ *                            (SF_SRC_OUTPUT_BF16, sf_forward_tracked) keep the row magnitude as
+ *                            bf16 in its first 2R bytes, and then need it 16-byte aligned
  *   words[R/32]      uint32  the mask: bit i of words[w] is row 32w+i
  *   active_rows[R]   int32   active rows, ascending; the first counts[0] are valid
  *   active_tiles[R/32] int32 tiles holding an active row, ascending; first counts[1] valid

@@ -173,6 +173,21 @@ SF_DEVICE uint16_t ld_nc_l2_64b_u16(const uint16_t *p)
 // Ask L2 to fetch the line holding p (no register result; the load that follows hits L2).
 SF_DEVICE void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
+// Element-wise max of eight bf16 values into p[0..7] (16-byte aligned), one reduction for all.
+// The row magnitudes reduced this way are non-negative and finite, so bf16 order is the order of
+// the bit patterns.
+SF_DEVICE void red_max_bf16x8(uint16_t *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    asm volatile("red.global.v4.bf16x2.max.noftz [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c),
+                 "r"(d) : "memory");
+}
+
+// The same for two bf16 values into p[0..1] (4-byte aligned).
+SF_DEVICE void red_max_bf16x2(uint16_t *p, uint16_t a, uint16_t b)
+{
+    asm volatile("red.global.v2.bf16.max.noftz [%0], {%1, %2};" ::"l"(p), "h"(a), "h"(b) : "memory");
+}
+
 SF_DEVICE void prefetch_tmap(const CUtensorMap *m)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");

@@ -314,11 +314,14 @@ forward_tracked_kernel(const __grid_constant__ FwdBatch b, uint32_t *status)
                 }
             }
             asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(128) : "memory");
-            {   // one thread per weight row of the half: the largest of the four warps' maxima
+            {   // one thread per weight row of the half: the largest of the four warps' maxima, into
+                // the mask's bf16 accumulator two rows at a time (the even lane of each pair)
                 const int c = (warp & 3) * 32 + lane;           // 0..127 over the half's 4 warps
                 const uint32_t m = max(max(colmax[half][0][c], colmax[half][1][c]),
                                        max(colmax[half][2][c], colmax[half][3][c]));
-                if (m && r0 + c < p.R) atomicMax(&p.accum[r0 + c], m << 16);
+                const uint32_t m_next = __shfl_down_sync(0xffffffffu, m, 1);
+                if ((lane & 1) == 0 && (m | m_next) && r0 + c < p.R)
+                    red_max_bf16x2(reinterpret_cast<uint16_t *>(p.accum) + r0 + c, (uint16_t)m, (uint16_t)m_next);
             }
             asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(128) : "memory");
         }
@@ -382,6 +385,7 @@ extern "C" int sf_forward_tracked(const sf_fwd_problem *probs, int n, uint32_t *
         const sf_fwd_problem &p = probs[i];
         const int R = p.mask.R;
         if (R <= 0 || (R & 31) || !p.mask.accum || p.T < 0 || p.C <= 0 || (p.C & 7)) return SF_ERR_ARG;
+        if (!aligned16(p.mask.accum)) return SF_ERR_ALIGN;     // the bf16 accumulator takes 16-byte reductions
         if (p.T > 0) {
             if (!p.A || !p.W || !p.Y || p.ld_a < p.C || p.ld_w < p.C || p.ld_y < R) return SF_ERR_ARG;
             if ((p.ld_a & 7) || (p.ld_w & 7) || (p.ld_y & 7) || !aligned16(p.A) || !aligned16(p.W) || !aligned16(p.Y))

@@ -90,6 +90,18 @@ __device__ __forceinline__ int find_mask_blk(const MaskBatch &b, int blk)
     return lo;
 }
 
+// An output source keeps the window's row magnitudes as bf16, two bytes per row at the start of
+// accum (16-byte aligned): the column-max pass reduces eight rows per instruction into it.
+// Counts (tokens) stay one uint32 per row. Either is read back as the uint32 the charge rule
+// takes: a count, or the magnitude widened to fp32 bits.
+__device__ __forceinline__ uint16_t *accum_bf16(const MaskDesc &d) { return reinterpret_cast<uint16_t *>(d.accum); }
+
+__device__ __forceinline__ uint32_t activity(const MaskDesc &d, int r)
+{
+    if (d.kind == SF_SRC_OUTPUT_BF16) return (uint32_t)accum_bf16(d)[r] << 16;
+    return d.kind == SF_SRC_HITS_U32 ? static_cast<const uint32_t *>(d.src)[r] : d.accum[r];
+}
+
 __global__ void __launch_bounds__(kAccumThreads)
 mask_accum_kernel(const __grid_constant__ MaskBatch b, uint32_t *status)
 {
@@ -178,15 +190,9 @@ mask_accum_kernel(const __grid_constant__ MaskBatch b, uint32_t *status)
         }
         set_status(status, SF_STATUS_NONFINITE);
     }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const uint32_t half = (mm[j] >> (16 * h)) & 0xFFFFu;
-            // widen bf16 magnitude to fp32 bits; non-negative floats order as unsigned ints
-            if (half) atomicMax(&d.accum[c0 + 2 * j + h], half << 16);
-        }
-    }
+    // the segment's maxima of the thread's eight columns into the mask's bf16 accumulator, one
+    // reduction for all eight (the packed pairs are in memory order)
+    if (mm[0] | mm[1] | mm[2] | mm[3]) red_max_bf16x8(accum_bf16(d) + c0, mm[0], mm[1], mm[2], mm[3]);
 }
 
 // The busiest row, the charge rule and the new words run over 2,048-row blocks (256 threads: a
@@ -217,7 +223,18 @@ mask_hmax_kernel(const __grid_constant__ MaskBatch b)
     const int r0 = (blockIdx.x - d.blk_begin) * kBlkRows;
     const int r1 = min(d.R, r0 + kBlkRows);
     uint32_t hmax = 0;
-    if ((reinterpret_cast<uintptr_t>(vals) & 15) == 0) {
+    if (d.kind == SF_SRC_OUTPUT_BF16) {       // bf16 magnitudes, eight rows per 16-byte load
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int u = 0; u < kBlkRows / (8 * kBlkThreads); ++u) {
+            const int r = r0 + 8 * (u * kBlkThreads + (int)threadIdx.x);
+            if (r < r1) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(accum_bf16(d) + r);
+                m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v.x, v.y), __vmaxu2(v.z, v.w)));
+            }
+        }
+        hmax = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+    } else if ((reinterpret_cast<uintptr_t>(vals) & 15) == 0) {
         // rows come in whole 32-row tiles, so each thread's four-row groups stay in the block
 #pragma unroll
         for (int u = 0; u < kBlkRows / (4 * kBlkThreads); ++u) {
@@ -260,7 +277,7 @@ __device__ __forceinline__ void charge_words(const MaskDesc &d, int w_begin, int
                 if (kind == SF_SRC_WORDS) {
                     hv[k] = src_u32[w];
                 } else {
-                    hv[k] = kind == SF_SRC_HITS_U32 ? src_u32[r] : d.accum[r];
+                    hv[k] = activity(d, r);
                     qv[k] = d.charge[r];
                 }
                 ow[k] = d.words[w];
@@ -280,7 +297,8 @@ __device__ __forceinline__ void charge_words(const MaskDesc &d, int w_begin, int
                 const float share = (H == 0.0f) ? 0.0f : __fdiv_rn(h, H);
                 const float q = __fadd_rn(__fmul_rn(0.5f, qv[k]), __fmul_rn(0.5f, share));
                 d.charge[r] = q;
-                if (kind != SF_SRC_HITS_U32) d.accum[r] = 0u;      // ready for the next window
+                if (kind == SF_SRC_OUTPUT_BF16) accum_bf16(d)[r] = 0;    // ready for the next window
+                else if (kind == SF_SRC_TOKENS) d.accum[r] = 0u;
                 act = q >= thr;
             }
             const bool was = (ow[k] >> lane) & 1u;
@@ -339,7 +357,16 @@ mask_finalize_kernel(const __grid_constant__ MaskBatch b, float thr, int fused, 
     griddep_wait();                           // the window's activity, or the charge pass's bit masks
     if (fused) {
         uint32_t hmax = 0;
-        if (d.kind != SF_SRC_WORDS) {
+        if (d.kind == SF_SRC_OUTPUT_BF16) {      // eight bf16 magnitudes per 16-byte load
+            const uint4 *v8 = reinterpret_cast<const uint4 *>(accum_bf16(d));
+            uint32_t m2 = 0;
+#pragma unroll 4
+            for (int k = tid; k < (R >> 3); k += kFinalizeThreads) {
+                const uint4 v = v8[k];
+                m2 = __vmaxu2(m2, __vmaxu2(__vmaxu2(v.x, v.y), __vmaxu2(v.z, v.w)));
+            }
+            hmax = max(m2 & 0xFFFFu, m2 >> 16) << 16;
+        } else if (d.kind != SF_SRC_WORDS) {
             const uint32_t *vals = d.kind == SF_SRC_HITS_U32 ? static_cast<const uint32_t *>(d.src) : d.accum;
 #pragma unroll 4
             for (int r = tid; r < R; r += kFinalizeThreads) hmax = max(hmax, vals[r]);
@@ -512,7 +539,7 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
             break;
         case SF_SRC_OUTPUT_BF16:
             if (s.n < 0 || (s.n > 0 && !s.ptr) || s.ld < m.R) return SF_ERR_ARG;
-            if ((s.ld & 7) || !aligned16(s.ptr)) return SF_ERR_ALIGN;
+            if ((s.ld & 7) || !aligned16(s.ptr) || !aligned16(m.accum)) return SF_ERR_ALIGN;
             break;
         case SF_SRC_HITS_U32:
         case SF_SRC_WORDS:
