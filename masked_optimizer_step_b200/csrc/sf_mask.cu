@@ -12,7 +12,8 @@
 // programmatic dependent launch:
 //   mask_accum_kernel     the window's activity into accum[] -- token histogram (integer
 //                         atomics), or the column absmax of Y (16-byte loads, packed u16 max,
-//                         one atomicMax per column and CTA). HBM-bound streaming pass.
+//                         per CTA one bf16 max-reduction per column, eight columns per
+//                         instruction). HBM-bound streaming pass.
 //   mask_hmax_kernel      the busiest row of each mask: 2,048-row blocks, one atomicMax each.
 //   mask_charge_kernel    the charge update and the new mask words, 2,048-row blocks, and per
 //                         32-row tile the rows that release a slot or need one.
@@ -564,7 +565,7 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
         // Token segment length of the column-absmax pass: 512 tokens, shortened (down to 32) when
         // the launch would otherwise give each SM fewer than ~2 CTAs, so that enough loads are in
         // flight to cover HBM latency (a lone projection has only R / 2048 column blocks). Each
-        // segment ends in one atomicMax per column, so shorter segments cost atomics: for one 7B
+        // segment ends in one max-reduction per column, so shorter segments cost atomics: for one 7B
         // layer at 4,096 tokens the pass measured fastest at ~2 CTAs per SM (4: +2 us, 8: +7 us,
         // 16: +35 us).
         int seg_tokens = kTokensPerSeg;
@@ -582,7 +583,7 @@ extern "C" int sf_mask_update_phase(const sf_mask *masks, const sf_mask_src *src
             // A large call gets shorter segments still, until it spans ~8 waves of resident CTAs:
             // the launch's last wave then idles fewer SMs (the 32-layer 7B step, 2,048 tokens:
             // 512 tokens 0.856 ms, 256 0.827, 128 0.813). Never below 128 tokens nor to more than
-            // 16 segments of the longest source: each segment ends in an atomicMax per column
+            // 16 segments of the longest source: each segment ends in a max-reduction per column
             // (64 tokens: 0.872 ms; one 7B layer at 4,096 tokens is fastest at 256).
             const long waves8 = 8L * accum_ctas_per_sm() * (sms > 0 ? sms : 148);
             int longest = 0;
