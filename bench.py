@@ -35,8 +35,8 @@ METRIC = "sparse step ms & active-row updates/s at 7B shape, 1% active; % of roo
 # capture), keyed by (layers, tokens, masks) of the workload it was captured on; a kernel or
 # workload not listed has none. Entries are removed whenever the kernel changes.
 TRAFFIC_PER_LAUNCH = {
-    "mask_accum_kernel": {(32, 2048, "scattered"): 16 * 348.6e6},
-    "dw_gather_kernel": {(32, 2048, "scattered"): 16 * 101.3e6},
+    "mask_accum_kernel": {(32, 2048, "scattered"): 16 * 348.5e6},
+    "dw_gather_kernel": {(32, 2048, "scattered"): 16 * 101.1e6},
 }
 TRAFFIC_NOTE = ("ncu DRAM bytes of the 2-layer case of this workload (profiles/kernels_2layer_dram.md) "
                 "scaled by 16 to 32 layers: one launch per step either way, bytes in proportion to the "
