@@ -144,3 +144,30 @@ def test_checkpoint_rejects(lib):
         assert call(name, C=24) == ARG           # rows copied in 16-byte vectors: C % 16 == 0
         assert call(name, cap=-1) == ARG
         assert call(name, count=None) == ARG
+
+
+def _mask_with(accum=P, R=256, cap=32):
+    return b.sf_mask(R, cap, P, accum, P, P, P, P, P, P, P, P)
+
+
+@pytest.mark.parametrize("case,accum,src,code", [
+    ("output source: accumulator not 16-byte aligned (bf16 rows, 16-byte reductions)", P + 4,
+     (b.SF_SRC_OUTPUT_BF16, 128, 256, P), ALIGN),
+    ("output source: Y not 16-byte aligned", P, (b.SF_SRC_OUTPUT_BF16, 128, 256, P + 2), ALIGN),
+    ("output source: row stride not a multiple of 8", P, (b.SF_SRC_OUTPUT_BF16, 128, 260, P), ALIGN),
+    ("output source: row stride below R", P, (b.SF_SRC_OUTPUT_BF16, 128, 128, P), ARG),
+    ("output source: negative token count", P, (b.SF_SRC_OUTPUT_BF16, -1, 256, P), ARG),
+    ("unknown source kind", P, (9, 128, 256, P), ARG),
+])
+def test_mask_update_rejects(lib, case, accum, src, code):
+    masks = (b.sf_mask * 1)(_mask_with(accum))
+    srcs = (b.sf_mask_src * 1)(b.sf_mask_src(*src))
+    assert lib.sf_mask_update(masks, srcs, 1, ctypes.c_float(0.01), None, None) == code, case
+
+
+def test_forward_tracked_rejects_a_misaligned_accumulator(lib):
+    # A [128 x 512], W [256 x 512], Y [128 x 256]; the mask's accumulator 4 bytes off
+    p = b.sf_fwd_problem(P, 512, P, 512, P, 256, 128, 512, _mask_with(P + 4))
+    assert lib.sf_forward_tracked((b.sf_fwd_problem * 1)(p), 1, None, None) == ALIGN
+    p = b.sf_fwd_problem(P, 512, P, 512, P + 8, 256, 128, 512, _mask_with(P))
+    assert lib.sf_forward_tracked((b.sf_fwd_problem * 1)(p), 1, None, None) == ALIGN
