@@ -233,10 +233,6 @@ update_kernel(const __grid_constant__ UpdBatch b, uint32_t *status)
         link_step();
         publish();
     }
-    // Everything above reads only what the masks' finalize left (lists, slots, step counts,
-    // scales); the gradients come from the kernel before this one on the stream, which this
-    // launch may overlap (programmatic dependent launch): wait for it here.
-    griddep_wait();
 
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
         __syncthreads();                 // this row's metadata is published; the shared row is free
@@ -510,22 +506,14 @@ extern "C" int sf_sparse_update(const sf_matrix *mats, int n_mats, const sf_adam
             d.pgrad = a.partner >= 0 ? mats[a.partner].grad : nullptr;
             d.prow_slot = a.partner >= 0 ? mats[a.partner].mask.row_slot : nullptr;
         }
-        // the launch may start while the kernel before it (the gradients' producer) finishes; the
-        // kernel waits for it before its first gradient read. It does not release its own
-        // successor early: the next window's finalize rewrites the slots this kernel reads.
-        cudaLaunchAttribute attr;
-        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr.val.programmaticStreamSerializationAllowed = 1;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(sms * per_sm);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem;
-        cfg.stream = st;
-        cfg.attrs = &attr;
-        cfg.numAttrs = 1;
-        const cudaError_t e = unroll == 2 ? cudaLaunchKernelEx(&cfg, update_kernel<2>, b, dev_status)
-                                          : cudaLaunchKernelEx(&cfg, update_kernel<1>, b, dev_status);
-        if (e != cudaSuccess || launch_status() != SF_OK) return SF_ERR_CUDA;
+        // A plain launch: the kernel reads the masks' lists and slots from its first instruction,
+        // and the call may directly follow the masks' finalize, which releases its successor
+        // early (programmatic dependent launch) for its own chained launches.
+        if (unroll == 2)
+            update_kernel<2><<<sms * per_sm, kThreads, smem, st>>>(b, dev_status);
+        else
+            update_kernel<1><<<sms * per_sm, kThreads, smem, st>>>(b, dev_status);
+        if (launch_status() != SF_OK) return SF_ERR_CUDA;
     }
     return SF_OK;
 }
