@@ -1,5 +1,6 @@
 """The full 7B-shaped model over 20 steps (the run the throughput figure is quoted on), with
-layers 0 and 31 and the embedding checked against the oracle at every step.
+layers 0 and 31 and the embedding checked against the oracle at every step; and the same model
+with rows clustered into whole 32-row tiles (the dW in tile mode) over 6 steps.
 
 Each step runs the same StepPlan calls as the benchmark (all 225 masks in one call, the masked
 dW of all 224 projections, the embedding-row gradient, one grouped update), alternating the two
@@ -29,9 +30,8 @@ from tests.gpu_helpers import DEV, check_slot_invariants, host, mask_host
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
-SEED, T, PRIOR, STEPS = 3, 2048, 20, 20
+SEED, T, PRIOR = 3, 2048, 20
 CHECK_LAYERS = (0, 31)
-DW_STEPS = (0, 9, 19)
 DW_TOL = 2e-3
 K = 32                                    # sampled rows per checked matrix
 
@@ -49,7 +49,9 @@ def _seeded_grad(step, j, R, C):
     return torch.randn((R, C), generator=gen, device=DEV, dtype=torch.float32).mul_(8.0)
 
 
-def test_twenty_steps_layers_0_and_31_and_embedding_follow_the_oracle():
+@pytest.mark.parametrize("kind,STEPS", [("scattered", 20), ("clustered", 6)])
+def test_steps_layers_0_and_31_and_embedding_follow_the_oracle(kind, STEPS):
+    DW_STEPS = (0, STEPS // 2 - 1, STEPS - 1)
     torch.cuda.set_device(0)
     torch.cuda.empty_cache()
     model = SparseModel(32, device=DEV)
@@ -62,8 +64,8 @@ def test_twenty_steps_layers_0_and_31_and_embedding_follow_the_oracle():
         R, C = p.mat.R, p.mat.C
         W = synth.weights_f32(synth.rng(SEED, "weights", 1000 + i), R, C)
         sf.sf_quantize_init(torch.from_numpy(W).to(DEV), p.mat)
-        c0 = synth.chosen_rows(SEED, p.layer, i, R, "scattered", 0)
-        c1 = synth.chosen_rows(SEED, p.layer, i, R, "scattered", 1)
+        c0 = synth.chosen_rows(SEED, p.layer, i, R, kind, 0)
+        c1 = synth.chosen_rows(SEED, p.layer, i, R, kind, 1)
         pick = np.unique(np.concatenate([c0[:20], np.setdiff1d(c1, c0)[:8],
                                          np.setdiff1d(np.arange(R), np.union1d(c0, c1))[:4]]))
         assert len(pick) <= K
@@ -73,7 +75,7 @@ def test_twenty_steps_layers_0_and_31_and_embedding_follow_the_oracle():
         subs[i] = orc.MatrixState(Wt)
         del W
     projs = [(p.layer, p.name, p.mat.R, p.mat.C, INPUT_OF[p.name]) for p in model.projs]
-    banks = [synth.step_bank(projs, T, "scattered", b, SEED, device=DEV) for b in (0, 1)]
+    banks = [synth.step_bank(projs, T, kind, b, SEED, device=DEV) for b in (0, 1)]
     toks = synth.token_stream(SEED, PRIOR + STEPS, T)
     tok_dev = torch.from_numpy(toks).to(DEV)
     emb_charge = np.zeros(model.emb.R, np.float32)
